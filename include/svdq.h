@@ -1,0 +1,203 @@
+/*
+ * svdq.h - C ABI of the B200 (sm_100a) SVDQuant W4A4 + low-rank linear layer.
+ *
+ * The layer computes (msModelSlim "SVDQuant Low-Rank Residual Quantization
+ * Algorithm Terminology Entry", section 2.3, the dual-path output equation,
+ * with the bias of the migration identity added):
+ *
+ *     Y = Q(X diag(s)^-1) Q(R) + (X diag(s)^-1 L1) L2 + b
+ *
+ * with s the smoothing factor of section 2.3 eq. 2, L1 L2 the rank-r truncated
+ * SVD of the migrated weight diag(s) W (section 2.2; eq. 3) and R the residual
+ * quantized to 4 bits per group along K ("SVDQuant: Absorbing Outliers by
+ * Low-Rank Components for 4-Bit Diffusion Models", abstract).
+ *
+ * Conventions for every call:
+ *  - All tensors are plain row-major device pointers unless a parameter says
+ *    "host". X is bf16 [M, K], W is bf16 [K, N] (Y = X W + b), Y is bf16 [M, N].
+ *    Device pointers must be 16-byte aligned.
+ *  - Ownership: the caller owns every pointer it passes (X, Y, W, bias, the
+ *    calibration statistic, LoRA factors, workspaces, the stream). The library
+ *    never frees them and keeps no reference after the call returns, except
+ *    that work queued on `stream` reads/writes them until it completes.
+ *    A layer handle owns its prepared device buffers; svdq_destroy frees them.
+ *  - Streams: `stream` is a cudaStream_t (NULL = legacy default stream). All
+ *    device work is queued on it; svdq_linear_forward and
+ *    svdq_quantize_activations never synchronize the host. A handle is used by
+ *    one stream at a time; svdq_attach_lora must be stream-ordered with the
+ *    forwards that precede it.
+ *  - Errors: every call returns an svdq_status and never aborts or throws.
+ *    svdq_last_error() returns a thread-local description of the last failure.
+ *    Launch failures come back as SVDQ_ERR_CUDA. A pipeline wait inside a
+ *    kernel that gives up (it never blocks forever) is reported by
+ *    svdq_device_status() as SVDQ_ERR_DEVICE_TIMEOUT.
+ *  - Shape limits: K a multiple of 128; N a multiple of 16; M >= 1;
+ *    1 <= rank (after any LoRA concatenation) <= 256 (section 2.6 recommends
+ *    rank <= 128; the larger limit leaves room for LoRA adapters); only 2-D
+ *    linear weights (section 2.6).
+ */
+#ifndef SVDQ_H_
+#define SVDQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(SVDQ_BUILD) && defined(__GNUC__)
+#define SVDQ_API __attribute__((visibility("default")))
+#else
+#define SVDQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,     /* bad pointer, shape, alignment or workspace size */
+  SVDQ_ERR_UNSUPPORTED = 2,     /* no sm_100 device, or a shape outside the limits above */
+  SVDQ_ERR_OOM = 3,             /* a device allocation of the library failed */
+  SVDQ_ERR_CUDA = 4,            /* a CUDA / cuSOLVER call or a kernel launch failed */
+  SVDQ_ERR_NUMERIC = 5,         /* the SVD did not converge or produced non-finite values */
+  SVDQ_ERR_DEVICE_TIMEOUT = 6   /* a kernel gave up a pipeline wait (see svdq_device_status) */
+} svdq_status;
+
+typedef enum {
+  SVDQ_INT4_G64 = 0,  /* symmetric INT4, 64 values per group along K, fp32 scale = amax/7 */
+  SVDQ_NVFP4_G16 = 1  /* E2M1 values, 16 per group along K, E4M3 group scale, fp32 tensor scale */
+} svdq_format;
+
+typedef struct {
+  int K;            /* input features (rows of W) */
+  int N;            /* output features (columns of W) */
+  int rank;         /* r of the truncated SVD, 1..256 */
+  float alpha;      /* migration strength of eq. 2, in [0, 1] */
+  float s_min;      /* lower clamp of s in eq. 2 (> 0; 1e-5 is the documented default) */
+  svdq_format fmt;  /* 4-bit format of Q(.) */
+} svdq_config;
+
+typedef struct svdq_layer* svdq_layer_t;
+
+typedef struct {
+  int K, N, rank;   /* rank includes attached LoRA adapters */
+  int rank_pad;     /* rank rounded up to a multiple of 32 (layout of the branch buffers) */
+  int fmt;          /* svdq_format */
+  float alpha;
+  float g_x;        /* NVFP4 static activation tensor scale (1 for INT4) */
+  float g_w;        /* NVFP4 residual tensor scale (1 for INT4) */
+  float t_scale;    /* factor applied to T before its bf16 store: 1 (INT4) or 1/(g_x g_w) (NVFP4) */
+} svdq_layer_info;
+
+/* Activation statistic A_scale of eq. 2 (section 2.3: per-channel absolute
+ * maximum of the activations) over a calibration batch.
+ *   X            device bf16 [M, K]
+ *   absmax_inout device float [K]; updated in place to max(absmax, max_m |X[m,k]|),
+ *                so several calibration batches can be folded in. Initialise
+ *                it to zeros before the first batch. */
+SVDQ_API svdq_status svdq_calibrate_absmax(const void* X, int M, int K, float* absmax_inout, void* stream);
+
+/* Offline preparation (section 2.1, in order: migrate, decompose, quantize):
+ *  1. W_scale[k] = max_n |W[k,n]| (the weight statistic of eq. 2, per input
+ *     channel); s = A_scale^alpha / W_scale^(1-alpha) computed in float64 on the
+ *     host (sqrt/sqrt for alpha = 0.5), rounded to float32, clamped at s_min
+ *     (s = 1 where a statistic is 0); inv_s = 1/s in float32.
+ *  2. W_hat = fp32(s_k W[k,n]) (eq. 1); float64 SVD of W_hat (cuSOLVER gesvd);
+ *     L1 = U_r, L2 = Sigma_r V_r^T, each column of L1 signed so that its
+ *     largest-magnitude entry is positive, both rounded to bf16.
+ *  3. R = fp32(W_hat - L1 L2) (float64 sums, j = 0..r-1 in order), quantized
+ *     per output column in groups of G along K.
+ *   W          device bf16 [K, N]
+ *   bias       device bf16 [N], or NULL for no bias
+ *   act_absmax device float [K] (from svdq_calibrate_absmax)
+ *   out        receives the new handle (NULL on failure)
+ * Synchronizes `stream` (the SVD's convergence flag is read on the host). */
+SVDQ_API svdq_status svdq_prepare_weights(const svdq_config* cfg, const void* W, const void* bias, const float* act_absmax,
+                                 void* stream, svdq_layer_t* out);
+
+/* As svdq_prepare_weights, with the bf16 factors given instead of computed
+ * (e.g. from an offline SVD): L1 device bf16 [K, rank], L2 device bf16
+ * [rank, N]. Steps 1 and 3 are unchanged. */
+SVDQ_API svdq_status svdq_prepare_weights_with_factors(const svdq_config* cfg, const void* W, const void* bias,
+                                              const float* act_absmax, const void* L1, const void* L2, void* stream,
+                                              svdq_layer_t* out);
+
+/* Bytes of workspace svdq_linear_forward needs for M rows. */
+SVDQ_API svdq_status svdq_workspace_size(svdq_layer_t layer, int M, size_t* bytes);
+
+/* The hot path: Y = Q(X diag(s)^-1) Q(R) + (X diag(s)^-1 L1) L2 + b, bf16 out.
+ * Two kernels on `stream`: (1) smoothing + group quantization of X + the
+ * down-projection T = x_hat L1 in one pass over X; (2) the 4-bit GEMM whose
+ * epilogue adds T L2 and the bias before a single bf16 store of Y.
+ *   X          device bf16 [M, K]
+ *   Y          device bf16 [M, N] (overwritten)
+ *   workspace  device buffer of at least svdq_workspace_size(layer, M) bytes,
+ *              256-byte aligned; its contents need no initialisation. */
+SVDQ_API svdq_status svdq_linear_forward(svdq_layer_t layer, const void* X, int M, void* Y, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/* Attaches a LoRA adapter Y += scale X A B to the low-rank branch without
+ * re-quantizing R (abstract: off-the-shelf LoRAs without re-quantization).
+ * The branch sees X diag(s)^-1, so L1' = [L1 | bf16(diag(s) A)] and
+ * L2' = [L2 ; bf16(scale B)]. The residual codes and scales are untouched.
+ * Adapters accumulate: each call appends r_l more columns.
+ *   A  device bf16 [K, r_l];  B  device bf16 [r_l, N];  1 <= rank + r_l <= 256.
+ * Synchronizes `stream` before freeing the previous branch buffers. */
+SVDQ_API svdq_status svdq_attach_lora(svdq_layer_t layer, const void* A, const void* B, int r_l, float scale, void* stream);
+
+/* The first kernel of the forward alone, into caller buffers, for inspection:
+ *   codes   INT4: uint8 [M_pad, K], the E4M3 encoding of each integer code
+ *                 (-8..7; exact). NVFP4: uint8 [M_pad, K/2], two E2M1 codes per
+ *                 byte, element 2j in bits 3:0.
+ *   scales  INT4: float [K/64][M_pad] (group scale amax/7, transposed).
+ *           NVFP4: uint8 E4M3 in 512-byte atoms, atom (m/128)*(K/64) + k/64,
+ *                  byte (m%32)*16 + ((m/32)%4)*4 + (k/16)%4.
+ *   T       bf16 [M_pad, rank_pad] = t_scale * (x_hat L1) (columns >= rank are 0)
+ * with M_pad = M rounded up to a multiple of 128 (rows >= M are zero codes). */
+SVDQ_API svdq_status svdq_quantize_activations(svdq_layer_t layer, const void* X, int M, void* codes, void* scales, void* T,
+                                      void* stream);
+
+/* Prepared weights in canonical layout, for checkpointing and inspection.
+ * With blob == NULL only *bytes is set. Otherwise *bytes must be at least the
+ * size and the blob (host memory) receives an svdq_blob_header followed by the
+ * sections at the offsets it lists. Synchronizes `stream`. */
+typedef struct {
+  uint32_t magic;     /* 0x51445653 ("SVDQ") */
+  uint32_t version;   /* 1 */
+  int32_t fmt, K, N, rank;
+  float alpha, g_x, g_w, reserved;
+  uint64_t off_s;       /* float [K] */
+  uint64_t off_inv_s;   /* float [K] */
+  uint64_t off_L1;      /* bf16 [K, rank] */
+  uint64_t off_L2;      /* bf16 [rank, N] */
+  uint64_t off_codes;   /* uint8 [N, K/2]: two 4-bit codes per byte, element 2j in bits 3:0;
+                           INT4 two's complement, NVFP4 E2M1 */
+  uint64_t off_scales;  /* INT4 float [N, K/64]; NVFP4 uint8 E4M3 [N, K/16] */
+  uint64_t off_bias;    /* bf16 [N] */
+  uint64_t total;
+} svdq_blob_header;
+
+SVDQ_API svdq_status svdq_export_weights(svdq_layer_t layer, void* blob, size_t* bytes, void* stream);
+
+SVDQ_API svdq_status svdq_layer_get_info(svdq_layer_t layer, svdq_layer_info* info);
+
+/* Reads and clears the layer's device status word (synchronizes `stream`):
+ * SVDQ_OK, or SVDQ_ERR_DEVICE_TIMEOUT if a kernel of this layer gave up a wait. */
+SVDQ_API svdq_status svdq_device_status(svdq_layer_t layer, void* stream);
+
+/* Frees the handle and its device buffers (synchronizes the device first). */
+SVDQ_API svdq_status svdq_destroy(svdq_layer_t layer);
+
+/* Thread-local message of the last failed call ("" if none). */
+SVDQ_API const char* svdq_last_error(void);
+
+/* Failure-detection self-test: launches a kernel that waits on a barrier no
+ * one arrives on, with the library's bounded wait shortened to limit_ns, and
+ * returns SVDQ_ERR_DEVICE_TIMEOUT when the wait gave up as designed (the
+ * context stays usable). Synchronizes `stream`. */
+SVDQ_API svdq_status svdq_selftest_bounded_wait(unsigned long long limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_H_ */

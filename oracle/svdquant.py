@@ -75,6 +75,7 @@ def smoothing_factors(a: np.ndarray, w: np.ndarray, alpha: float, s_min: float =
     at s_min; a channel whose activation or weight statistic is 0 keeps s = 1.
     inv_s = 1 / s in float32.
     """
+    alpha = float(F32(alpha))  # alpha is a float32 parameter of the layer
     a64 = np.asarray(a, dtype=np.float64)
     w64 = np.asarray(w, dtype=np.float64)
     dead = (a64 == 0) | (w64 == 0)

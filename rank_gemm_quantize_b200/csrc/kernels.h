@@ -1,0 +1,70 @@
+// Internal launch interfaces of the SVDQuant kernels (not part of the C ABI).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace svdq {
+
+// ---------------------------------------------------------------- K1
+struct ActQuantParams {
+  const __nv_bfloat16* X;  // [M, K] row-major
+  int M, K, M_pad;         // M_pad = roundup(M, 128)
+  const float* inv_s;      // [K]
+  const __nv_bfloat16* L1T;  // [RP, K]: transposed, zero-padded down-projection factor
+  uint8_t* codes;          // INT4: [M_pad, K] E4M3 bytes of the integer codes; NVFP4: [M_pad, K/2] packed E2M1
+  void* scales;            // INT4: float [K/64][M_pad]; NVFP4: scale-factor atoms [M_pad/128][K/64][512]
+  __nv_bfloat16* T;        // [M_pad, RP] bf16, multiplied by t_scale
+  float g_x;               // NVFP4 activation tensor scale
+  float denom;             // NVFP4: fp32(6 * g_x)
+  float t_scale;           // 1 (INT4) or 1 / (g_x g_w) (NVFP4)
+};
+cudaError_t launch_act_quant(const ActQuantParams& p, int fmt, int rp, cudaStream_t stream);
+
+// ---------------------------------------------------------------- GEMMs
+struct GemmParams {
+  int M, N, K, RP;
+  __nv_bfloat16* Y;            // [M, N]
+  const __nv_bfloat16* bias;   // [N]
+  const void* sa;              // activation scales (layout of ActQuantParams::scales)
+  const void* sb;              // weight scales: INT4 float [K/64][N_pad]; NVFP4 atoms [N_pad/128][K/64][512]
+  int M_pad, N_pad;
+  float out_scale;             // NVFP4: g_x g_w; INT4: 1
+  int* status;                 // device status word (kDevTimeout on a given-up wait)
+};
+struct GemmMaps {
+  CUtensorMap a;   // activation codes
+  CUtensorMap b;   // weight codes
+  CUtensorMap t;   // T [M_pad, RP] bf16
+  CUtensorMap l2;  // L2T [N_pad, RP] bf16
+};
+cudaError_t launch_gemm_nvfp4(const GemmParams& p, const GemmMaps& maps, cudaStream_t stream);
+cudaError_t launch_gemm_int4(const GemmParams& p, const GemmMaps& maps, cudaStream_t stream);
+
+// ---------------------------------------------------------------- prepare
+cudaError_t launch_absmax_rows(const __nv_bfloat16* W, int K, int N, float* out, cudaStream_t s);
+cudaError_t launch_absmax_cols(const __nv_bfloat16* X, int M, int K, float* running_max, cudaStream_t s);
+cudaError_t launch_migrate(const __nv_bfloat16* W, const float* s_k, int K, int N, float* W_hat, cudaStream_t st);
+cudaError_t launch_to_f64_colmajor(const float* W_hat, int K, int N, bool transpose, double* out, cudaStream_t st);
+cudaError_t launch_factors_from_svd(const double* U, const double* S, const double* VT, int K, int N, int rank,
+                                    bool wt, int ldu, int ldvt, __nv_bfloat16* L1, __nv_bfloat16* L2,
+                                    cudaStream_t st);
+cudaError_t launch_residual(const float* W_hat, const __nv_bfloat16* L1, const __nv_bfloat16* L2, int K, int N,
+                            int rank, float* R, cudaStream_t st);
+cudaError_t launch_absmax_all(const float* R, size_t n, unsigned int* out_bits, cudaStream_t st);
+cudaError_t launch_quant_weight_int4(const float* R, int K, int N, int N_pad, uint8_t* codes8, float* sw,
+                                     cudaStream_t st);
+cudaError_t launch_quant_weight_nvfp4(const float* R, int K, int N, int N_pad, const unsigned int* amax_bits,
+                                      uint8_t* codes4, uint8_t* sf_atoms, float* g_w_out, cudaStream_t st);
+cudaError_t launch_build_branch(const __nv_bfloat16* L1, const __nv_bfloat16* L2, int K, int N, int rank, int RP,
+                                int N_pad, __nv_bfloat16* L1T, __nv_bfloat16* L2T, cudaStream_t st);
+cudaError_t launch_lora_concat(const __nv_bfloat16* L1T_old, const __nv_bfloat16* L2T_old, int K, int N, int N_pad,
+                               int rank_old, int RP_old, const float* s_k, const __nv_bfloat16* A,
+                               const __nv_bfloat16* B, int r_l, float scale, int RP_new, __nv_bfloat16* L1T,
+                               __nv_bfloat16* L2T, cudaStream_t st);
+cudaError_t launch_wait_selftest(int* status, unsigned long long limit_ns, cudaStream_t st);
+
+}  // namespace svdq

@@ -1,0 +1,719 @@
+// Host side of the C ABI: argument checks, the layer handle, the offline
+// preparation pipeline (cuSOLVER float64 SVD between our own kernels), the
+// forward's two launches, LoRA attach, export to the canonical layout.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <cudaTypedefs.h>
+#include <cusolverDn.h>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace svdq;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+svdq_status fail(svdq_status st, const std::string& msg) {
+  g_last_error = msg;
+  return st;
+}
+
+#define CUDA_TRY(expr)                                                                              \
+  do {                                                                                              \
+    cudaError_t e__ = (expr);                                                                       \
+    if (e__ != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string(#expr) + ": " + cudaGetErrorString(e__)); \
+  } while (0)
+
+inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D tiled tensor map: inner dimension contiguous, rows row_bytes apart.
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  auto enc = get_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+constexpr int kGemmBN = 128;
+
+struct WsLayout {
+  int M_pad;
+  size_t codes, scales, T, total;
+};
+
+}  // namespace
+
+struct svdq_layer {
+  int device = 0;
+  svdq_config cfg{};
+  int K = 0, N = 0, N_pad = 0, rank = 0, RP = 0;
+  int fmt = 0;
+  float g_x = 1.f, g_w = 1.f, gxgw = 1.f, t_scale = 1.f, denom = 6.f;
+  float* s = nullptr;
+  float* inv_s = nullptr;
+  __nv_bfloat16* L1T = nullptr;  // [RP, K]
+  __nv_bfloat16* L2T = nullptr;  // [N_pad, RP]
+  __nv_bfloat16* bias = nullptr; // [N]
+  uint8_t* wcodes = nullptr;     // INT4 [N_pad, K] E4M3 bytes; NVFP4 [N_pad, K/2]
+  void* wscales = nullptr;       // INT4 float [K/64][N_pad]; NVFP4 atoms [N_pad/128][K/64][512]
+  int* status = nullptr;         // device status word
+  CUtensorMap map_b{}, map_l2{};
+  // per-workspace maps, rebuilt when the workspace pointer or M changes
+  const void* ws_key = nullptr;
+  int M_key = -1;
+  CUtensorMap map_a{}, map_t{};
+};
+
+namespace {
+
+WsLayout ws_layout(const svdq_layer* h, int M) {
+  WsLayout w{};
+  w.M_pad = round_up(M, 128);
+  const size_t cbytes = h->fmt == SVDQ_INT4_G64 ? static_cast<size_t>(w.M_pad) * h->K
+                                                : static_cast<size_t>(w.M_pad) * (h->K / 2);
+  const size_t sbytes = h->fmt == SVDQ_INT4_G64 ? static_cast<size_t>(h->K / 64) * w.M_pad * 4
+                                                : static_cast<size_t>(w.M_pad / 128) * (h->K / 64) * 512;
+  w.codes = 0;
+  w.scales = align256(cbytes);
+  w.T = w.scales + align256(sbytes);
+  w.total = w.T + align256(static_cast<size_t>(w.M_pad) * h->RP * 2);
+  return w;
+}
+
+svdq_status check_device() {
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  int major = 0, minor = 0;
+  CUDA_TRY(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+  CUDA_TRY(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+  if (major != 10 || minor != 0) return fail(SVDQ_ERR_UNSUPPORTED, "svdq needs an sm_100 (B200-class) device");
+  return SVDQ_OK;
+}
+
+svdq_status check_cfg(const svdq_config* cfg) {
+  if (!cfg) return fail(SVDQ_ERR_INVALID_ARG, "cfg is NULL");
+  if (cfg->K <= 0 || cfg->K % 128) return fail(SVDQ_ERR_INVALID_ARG, "K must be a positive multiple of 128");
+  if (cfg->N <= 0 || cfg->N % 16) return fail(SVDQ_ERR_INVALID_ARG, "N must be a positive multiple of 16");
+  if (cfg->rank < 1 || cfg->rank > 256) return fail(SVDQ_ERR_INVALID_ARG, "rank must be in [1, 256]");
+  if (cfg->rank > std::min(cfg->K, cfg->N)) return fail(SVDQ_ERR_INVALID_ARG, "rank exceeds min(K, N)");
+  if (!(cfg->alpha >= 0.f && cfg->alpha <= 1.f)) return fail(SVDQ_ERR_INVALID_ARG, "alpha must be in [0, 1]");
+  if (!(cfg->s_min > 0.f) || !std::isfinite(cfg->s_min)) return fail(SVDQ_ERR_INVALID_ARG, "s_min must be > 0");
+  if (cfg->fmt != SVDQ_INT4_G64 && cfg->fmt != SVDQ_NVFP4_G16) return fail(SVDQ_ERR_INVALID_ARG, "unknown format");
+  return SVDQ_OK;
+}
+
+template <class T>
+svdq_status dalloc(T** p, size_t bytes) {
+  *p = nullptr;
+  if (cudaMalloc(reinterpret_cast<void**>(p), std::max<size_t>(bytes, 256)) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(SVDQ_ERR_OOM, "cudaMalloc of " + std::to_string(bytes) + " bytes failed");
+  }
+  return SVDQ_OK;
+}
+
+void free_layer(svdq_layer* h) {
+  if (!h) return;
+  cudaFree(h->s);
+  cudaFree(h->inv_s);
+  cudaFree(h->L1T);
+  cudaFree(h->L2T);
+  cudaFree(h->bias);
+  cudaFree(h->wcodes);
+  cudaFree(h->wscales);
+  cudaFree(h->status);
+  delete h;
+}
+
+svdq_status build_static_maps(svdq_layer* h) {
+  const bool i4 = h->fmt == SVDQ_INT4_G64;
+  const uint64_t row = i4 ? h->K : h->K / 2;
+  if (!make_map(&h->map_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, row, h->N_pad, row, 128, kGemmBN,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (weight codes) failed");
+  if (!make_map(&h->map_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->L2T, h->RP, h->N_pad, static_cast<uint64_t>(h->RP) * 2,
+                32, kGemmBN, CU_TENSOR_MAP_SWIZZLE_64B))
+    return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (L2) failed");
+  h->M_key = -1;
+  h->ws_key = nullptr;
+  return SVDQ_OK;
+}
+
+// Host part of eq. 2 (float64, one rounding to float32), plus the NVFP4 static
+// activation tensor scale.
+void smoothing_host(const std::vector<float>& a, const std::vector<float>& w, float alpha, float s_min,
+                    std::vector<float>& s, std::vector<float>& inv_s) {
+  const size_t K = a.size();
+  s.resize(K);
+  inv_s.resize(K);
+  for (size_t k = 0; k < K; ++k) {
+    double sk;
+    if (a[k] == 0.f || w[k] == 0.f) {
+      sk = 1.0;
+    } else if (alpha == 0.5f) {
+      sk = std::sqrt(static_cast<double>(a[k])) / std::sqrt(static_cast<double>(w[k]));
+    } else {
+      sk = std::pow(static_cast<double>(a[k]), static_cast<double>(alpha)) /
+           std::pow(static_cast<double>(w[k]), 1.0 - static_cast<double>(alpha));
+    }
+    const float f = std::max(static_cast<float>(sk), s_min);  // s >= s_min for every channel
+    s[k] = f;
+    inv_s[k] = 1.0f / f;
+  }
+}
+
+float nvfp4_tensor_scale_host(float amax) {
+  if (amax == 0.f) return 1.0f;
+  volatile float d = 2688.0f;
+  return amax / d;
+}
+
+// Steps shared by both prepare entry points once L1 [K, rank] and L2 [rank, N]
+// (bf16, device) exist: residual, quantization, branch layout.
+svdq_status finish_prepare(svdq_layer* h, const float* W_hat, const __nv_bfloat16* L1, const __nv_bfloat16* L2,
+                           cudaStream_t st) {
+  const int K = h->K, N = h->N;
+  float* R = nullptr;
+  svdq_status e = dalloc(&R, static_cast<size_t>(K) * N * 4);
+  if (e) return e;
+  auto cleanup = [&] { cudaFree(R); };
+  if (launch_residual(W_hat, L1, L2, K, N, h->rank, R, st) != cudaSuccess) {
+    cleanup();
+    return fail(SVDQ_ERR_CUDA, "residual kernel launch failed");
+  }
+  if (h->fmt == SVDQ_INT4_G64) {
+    if ((e = dalloc(&h->wcodes, static_cast<size_t>(h->N_pad) * K))) return cleanup(), e;
+    if ((e = dalloc(reinterpret_cast<float**>(&h->wscales), static_cast<size_t>(K / 64) * h->N_pad * 4))) return cleanup(), e;
+    cudaMemsetAsync(h->wcodes, 0, static_cast<size_t>(h->N_pad) * K, st);
+    cudaMemsetAsync(h->wscales, 0, static_cast<size_t>(K / 64) * h->N_pad * 4, st);
+    if (launch_quant_weight_int4(R, K, N, h->N_pad, h->wcodes, static_cast<float*>(h->wscales), st) != cudaSuccess)
+      return cleanup(), fail(SVDQ_ERR_CUDA, "weight quantization launch failed");
+  } else {
+    unsigned int* amax = nullptr;
+    float* gw_dev = nullptr;
+    if ((e = dalloc(&h->wcodes, static_cast<size_t>(h->N_pad) * K / 2))) return cleanup(), e;
+    if ((e = dalloc(reinterpret_cast<uint8_t**>(&h->wscales), static_cast<size_t>(h->N_pad / 128) * (K / 64) * 512)))
+      return cleanup(), e;
+    if ((e = dalloc(&amax, 16))) return cleanup(), e;
+    gw_dev = reinterpret_cast<float*>(amax) + 1;
+    cudaMemsetAsync(h->wcodes, 0, static_cast<size_t>(h->N_pad) * K / 2, st);
+    cudaMemsetAsync(h->wscales, 0, static_cast<size_t>(h->N_pad / 128) * (K / 64) * 512, st);
+    cudaMemsetAsync(amax, 0, 16, st);
+    if (launch_absmax_all(R, static_cast<size_t>(K) * N, amax, st) != cudaSuccess ||
+        launch_quant_weight_nvfp4(R, K, N, h->N_pad, amax, h->wcodes, static_cast<uint8_t*>(h->wscales), gw_dev, st) !=
+            cudaSuccess) {
+      cudaFree(amax);
+      return cleanup(), fail(SVDQ_ERR_CUDA, "weight quantization launch failed");
+    }
+    float gw = 1.f;
+    cudaError_t ce = cudaMemcpyAsync(&gw, gw_dev, 4, cudaMemcpyDeviceToHost, st);
+    if (ce == cudaSuccess) ce = cudaStreamSynchronize(st);
+    cudaFree(amax);
+    if (ce != cudaSuccess) return cleanup(), fail(SVDQ_ERR_CUDA, cudaGetErrorString(ce));
+    h->g_w = gw;
+  }
+  // branch buffers
+  if ((e = dalloc(&h->L1T, static_cast<size_t>(h->RP) * K * 2))) return cleanup(), e;
+  if ((e = dalloc(&h->L2T, static_cast<size_t>(h->N_pad) * h->RP * 2))) return cleanup(), e;
+  if (launch_build_branch(L1, L2, K, N, h->rank, h->RP, h->N_pad, h->L1T, h->L2T, st) != cudaSuccess)
+    return cleanup(), fail(SVDQ_ERR_CUDA, "branch layout launch failed");
+  cudaError_t ce = cudaStreamSynchronize(st);
+  cleanup();
+  if (ce != cudaSuccess) return fail(SVDQ_ERR_CUDA, cudaGetErrorString(ce));
+  if (h->fmt == SVDQ_NVFP4_G16) {
+    h->gxgw = h->g_x * h->g_w;
+    h->t_scale = 1.0f / h->gxgw;
+  } else {
+    h->gxgw = 1.f;
+    h->t_scale = 1.f;
+  }
+  return build_static_maps(h);
+}
+
+// Steps 1 (statistics, eq. 2) and the migration of eq. 1.
+svdq_status start_prepare(const svdq_config* cfg, const void* W, const void* bias, const float* act_absmax,
+                          cudaStream_t st, svdq_layer** out_h, float** W_hat_out) {
+  svdq_status e;
+  if ((e = check_device())) return e;
+  if ((e = check_cfg(cfg))) return e;
+  if (!W || !act_absmax) return fail(SVDQ_ERR_INVALID_ARG, "W and act_absmax must not be NULL");
+  if (!aligned16(W) || (bias && !aligned16(bias)) || !aligned16(act_absmax))
+    return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  svdq_layer* h = new svdq_layer();
+  cudaGetDevice(&h->device);
+  h->cfg = *cfg;
+  h->K = cfg->K;
+  h->N = cfg->N;
+  h->N_pad = round_up(cfg->N, 128);
+  h->rank = cfg->rank;
+  h->RP = round_up(cfg->rank, 32);
+  h->fmt = cfg->fmt;
+  const int K = h->K, N = h->N;
+  auto bail = [&](svdq_status s) {
+    free_layer(h);
+    return s;
+  };
+  if ((e = dalloc(&h->s, K * 4)) || (e = dalloc(&h->inv_s, K * 4)) || (e = dalloc(&h->bias, N * 2)) ||
+      (e = dalloc(&h->status, 16)))
+    return bail(e);
+  cudaMemsetAsync(h->status, 0, 16, st);
+  if (bias)
+    cudaMemcpyAsync(h->bias, bias, N * 2, cudaMemcpyDeviceToDevice, st);
+  else
+    cudaMemsetAsync(h->bias, 0, N * 2, st);
+
+  float* wstat = nullptr;
+  if ((e = dalloc(&wstat, K * 4))) return bail(e);
+  if (launch_absmax_rows(static_cast<const __nv_bfloat16*>(W), K, N, wstat, st) != cudaSuccess) {
+    cudaFree(wstat);
+    return bail(fail(SVDQ_ERR_CUDA, "absmax kernel launch failed"));
+  }
+  std::vector<float> a(K), w(K), s, inv_s;
+  cudaError_t ce = cudaMemcpyAsync(a.data(), act_absmax, K * 4, cudaMemcpyDeviceToHost, st);
+  if (ce == cudaSuccess) ce = cudaMemcpyAsync(w.data(), wstat, K * 4, cudaMemcpyDeviceToHost, st);
+  if (ce == cudaSuccess) ce = cudaStreamSynchronize(st);
+  cudaFree(wstat);
+  if (ce != cudaSuccess) return bail(fail(SVDQ_ERR_CUDA, cudaGetErrorString(ce)));
+  for (int k = 0; k < K; ++k)
+    if (!(a[k] >= 0.f) || !std::isfinite(a[k])) return bail(fail(SVDQ_ERR_INVALID_ARG, "act_absmax must be finite and >= 0"));
+  smoothing_host(a, w, cfg->alpha, cfg->s_min, s, inv_s);
+  if (cfg->fmt == SVDQ_NVFP4_G16) {
+    float amax_x = 0.f;
+    for (int k = 0; k < K; ++k) {
+      volatile float prod = a[k] * inv_s[k];
+      amax_x = std::max(amax_x, static_cast<float>(prod));
+    }
+    h->g_x = nvfp4_tensor_scale_host(amax_x);
+    volatile float six = 6.0f;
+    h->denom = six * h->g_x;
+  }
+  ce = cudaMemcpyAsync(h->s, s.data(), K * 4, cudaMemcpyHostToDevice, st);
+  if (ce == cudaSuccess) ce = cudaMemcpyAsync(h->inv_s, inv_s.data(), K * 4, cudaMemcpyHostToDevice, st);
+  if (ce != cudaSuccess) return bail(fail(SVDQ_ERR_CUDA, cudaGetErrorString(ce)));
+  float* W_hat = nullptr;
+  if ((e = dalloc(&W_hat, static_cast<size_t>(K) * N * 4))) return bail(e);
+  if (launch_migrate(static_cast<const __nv_bfloat16*>(W), h->s, K, N, W_hat, st) != cudaSuccess) {
+    cudaFree(W_hat);
+    return bail(fail(SVDQ_ERR_CUDA, "migrate kernel launch failed"));
+  }
+  ce = cudaStreamSynchronize(st);
+  if (ce != cudaSuccess) {
+    cudaFree(W_hat);
+    return bail(fail(SVDQ_ERR_CUDA, cudaGetErrorString(ce)));
+  }
+  *out_h = h;
+  *W_hat_out = W_hat;
+  return SVDQ_OK;
+}
+
+// Truncated SVD of W_hat with cuSOLVER (float64 gesvd on whichever
+// orientation has m >= n), then L1, L2 in bf16.
+svdq_status svd_factors(svdq_layer* h, const float* W_hat, __nv_bfloat16* L1, __nv_bfloat16* L2, cudaStream_t st) {
+  const int K = h->K, N = h->N;
+  const bool wt = N >= K;  // SVD of W_hat^T (N x K) when N >= K, else of W_hat (K x N)
+  const int m = wt ? N : K, n = wt ? K : N;
+  double *A = nullptr, *S = nullptr, *U = nullptr, *VT = nullptr, *work = nullptr, *rwork = nullptr;
+  int* info = nullptr;
+  svdq_status e = SVDQ_OK;
+  cusolverDnHandle_t sh = nullptr;
+  auto cleanup = [&] {
+    cudaFree(A);
+    cudaFree(S);
+    cudaFree(U);
+    cudaFree(VT);
+    cudaFree(work);
+    cudaFree(rwork);
+    cudaFree(info);
+    if (sh) cusolverDnDestroy(sh);
+  };
+  if ((e = dalloc(&A, static_cast<size_t>(m) * n * 8)) || (e = dalloc(&S, static_cast<size_t>(n) * 8)) ||
+      (e = dalloc(&U, static_cast<size_t>(m) * n * 8)) || (e = dalloc(&VT, static_cast<size_t>(n) * n * 8)) ||
+      (e = dalloc(&rwork, static_cast<size_t>(n) * 8)) || (e = dalloc(&info, 16)))
+    return cleanup(), e;
+  if (launch_to_f64_colmajor(W_hat, K, N, !wt, A, st) != cudaSuccess)
+    return cleanup(), fail(SVDQ_ERR_CUDA, "layout kernel launch failed");
+  if (cusolverDnCreate(&sh) != CUSOLVER_STATUS_SUCCESS) return cleanup(), fail(SVDQ_ERR_CUDA, "cusolverDnCreate failed");
+  cusolverDnSetStream(sh, st);
+  int lwork = 0;
+  if (cusolverDnDgesvd_bufferSize(sh, m, n, &lwork) != CUSOLVER_STATUS_SUCCESS)
+    return cleanup(), fail(SVDQ_ERR_CUDA, "gesvd_bufferSize failed");
+  if ((e = dalloc(&work, static_cast<size_t>(lwork) * 8))) return cleanup(), e;
+  signed char jobu = 'S', jobvt = 'S';
+  if (cusolverDnDgesvd(sh, jobu, jobvt, m, n, A, m, S, U, m, VT, n, work, lwork, rwork, info) !=
+      CUSOLVER_STATUS_SUCCESS)
+    return cleanup(), fail(SVDQ_ERR_CUDA, "gesvd failed to launch");
+  int hinfo = 0;
+  cudaError_t ce = cudaMemcpyAsync(&hinfo, info, 4, cudaMemcpyDeviceToHost, st);
+  if (ce == cudaSuccess) ce = cudaStreamSynchronize(st);
+  if (ce != cudaSuccess) return cleanup(), fail(SVDQ_ERR_CUDA, cudaGetErrorString(ce));
+  if (hinfo != 0) return cleanup(), fail(SVDQ_ERR_NUMERIC, "gesvd did not converge (info=" + std::to_string(hinfo) + ")");
+  if (launch_factors_from_svd(U, S, VT, K, N, h->rank, wt, m, n, L1, L2, st) != cudaSuccess)
+    return cleanup(), fail(SVDQ_ERR_CUDA, "factor kernel launch failed");
+  ce = cudaStreamSynchronize(st);
+  cleanup();
+  if (ce != cudaSuccess) return fail(SVDQ_ERR_CUDA, cudaGetErrorString(ce));
+  return SVDQ_OK;
+}
+
+svdq_status launch_k1(svdq_layer* h, const void* X, int M, uint8_t* codes, void* scales, __nv_bfloat16* T,
+                      cudaStream_t st) {
+  ActQuantParams p{};
+  p.X = static_cast<const __nv_bfloat16*>(X);
+  p.M = M;
+  p.K = h->K;
+  p.M_pad = round_up(M, 128);
+  p.inv_s = h->inv_s;
+  p.L1T = h->L1T;
+  p.codes = codes;
+  p.scales = scales;
+  p.T = T;
+  p.g_x = h->g_x;
+  p.denom = h->denom;
+  p.t_scale = h->t_scale;
+  cudaError_t e = launch_act_quant(p, h->fmt, h->RP, st);
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("activation kernel: ") + cudaGetErrorString(e));
+  return SVDQ_OK;
+}
+
+svdq_status check_layer(svdq_layer* h) {
+  if (!h) return fail(SVDQ_ERR_INVALID_ARG, "layer is NULL");
+  return SVDQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* svdq_last_error(void) { return g_last_error.c_str(); }
+
+svdq_status svdq_calibrate_absmax(const void* X, int M, int K, float* absmax_inout, void* stream) {
+  if (!X || !absmax_inout || M < 1 || K < 1) return fail(SVDQ_ERR_INVALID_ARG, "bad calibration arguments");
+  if (launch_absmax_cols(static_cast<const __nv_bfloat16*>(X), M, K, absmax_inout, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return fail(SVDQ_ERR_CUDA, "calibration kernel launch failed");
+  return SVDQ_OK;
+}
+
+svdq_status svdq_prepare_weights(const svdq_config* cfg, const void* W, const void* bias, const float* act_absmax,
+                                 void* stream, svdq_layer_t* out) {
+  if (!out) return fail(SVDQ_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  svdq_layer* h = nullptr;
+  float* W_hat = nullptr;
+  svdq_status e = start_prepare(cfg, W, bias, act_absmax, st, &h, &W_hat);
+  if (e) return e;
+  __nv_bfloat16 *L1 = nullptr, *L2 = nullptr;
+  if ((e = dalloc(&L1, static_cast<size_t>(h->K) * h->rank * 2)) ||
+      (e = dalloc(&L2, static_cast<size_t>(h->rank) * h->N * 2)) || (e = svd_factors(h, W_hat, L1, L2, st)) ||
+      (e = finish_prepare(h, W_hat, L1, L2, st))) {
+    cudaFree(L1);
+    cudaFree(L2);
+    cudaFree(W_hat);
+    free_layer(h);
+    return e;
+  }
+  cudaFree(L1);
+  cudaFree(L2);
+  cudaFree(W_hat);
+  *out = h;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_prepare_weights_with_factors(const svdq_config* cfg, const void* W, const void* bias,
+                                              const float* act_absmax, const void* L1, const void* L2, void* stream,
+                                              svdq_layer_t* out) {
+  if (!out) return fail(SVDQ_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (!L1 || !L2) return fail(SVDQ_ERR_INVALID_ARG, "L1 and L2 must not be NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  svdq_layer* h = nullptr;
+  float* W_hat = nullptr;
+  svdq_status e = start_prepare(cfg, W, bias, act_absmax, st, &h, &W_hat);
+  if (e) return e;
+  e = finish_prepare(h, W_hat, static_cast<const __nv_bfloat16*>(L1), static_cast<const __nv_bfloat16*>(L2), st);
+  cudaFree(W_hat);
+  if (e) {
+    free_layer(h);
+    return e;
+  }
+  *out = h;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_workspace_size(svdq_layer_t h, int M, size_t* bytes) {
+  if (check_layer(h)) return SVDQ_ERR_INVALID_ARG;
+  if (!bytes || M < 1) return fail(SVDQ_ERR_INVALID_ARG, "bad workspace query");
+  *bytes = ws_layout(h, M).total;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_linear_forward(svdq_layer_t h, const void* X, int M, void* Y, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  if (check_layer(h)) return SVDQ_ERR_INVALID_ARG;
+  if (!X || !Y || !workspace || M < 1) return fail(SVDQ_ERR_INVALID_ARG, "NULL pointer or M < 1");
+  if (!aligned16(X) || !aligned16(Y) || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return fail(SVDQ_ERR_INVALID_ARG, "X/Y must be 16-byte and the workspace 256-byte aligned");
+  const WsLayout w = ws_layout(h, M);
+  if (ws_bytes < w.total) return fail(SVDQ_ERR_INVALID_ARG, "workspace too small");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  uint8_t* codes = base + w.codes;
+  void* scales = base + w.scales;
+  __nv_bfloat16* T = reinterpret_cast<__nv_bfloat16*>(base + w.T);
+  svdq_status e = launch_k1(h, X, M, codes, scales, T, st);
+  if (e) return e;
+  if (h->ws_key != workspace || h->M_key != M) {
+    const bool i4 = h->fmt == SVDQ_INT4_G64;
+    const uint64_t row = i4 ? h->K : h->K / 2;
+    if (!make_map(&h->map_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, row, w.M_pad, row, 128, 128,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&h->map_t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, h->RP, w.M_pad, static_cast<uint64_t>(h->RP) * 2, 32,
+                  128, CU_TENSOR_MAP_SWIZZLE_64B))
+      return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (activations) failed");
+    h->ws_key = workspace;
+    h->M_key = M;
+  }
+  GemmParams p{};
+  p.M = M;
+  p.N = h->N;
+  p.K = h->K;
+  p.RP = h->RP;
+  p.Y = static_cast<__nv_bfloat16*>(Y);
+  p.bias = h->bias;
+  p.sa = scales;
+  p.sb = h->wscales;
+  p.M_pad = w.M_pad;
+  p.N_pad = h->N_pad;
+  p.out_scale = h->gxgw;
+  p.status = h->status;
+  GemmMaps maps;
+  maps.a = h->map_a;
+  maps.b = h->map_b;
+  maps.t = h->map_t;
+  maps.l2 = h->map_l2;
+  cudaError_t ce = h->fmt == SVDQ_INT4_G64 ? launch_gemm_int4(p, maps, st) : launch_gemm_nvfp4(p, maps, st);
+  if (ce != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("GEMM kernel: ") + cudaGetErrorString(ce));
+  return SVDQ_OK;
+}
+
+svdq_status svdq_quantize_activations(svdq_layer_t h, const void* X, int M, void* codes, void* scales, void* T,
+                                      void* stream) {
+  if (check_layer(h)) return SVDQ_ERR_INVALID_ARG;
+  if (!X || !codes || !scales || !T || M < 1) return fail(SVDQ_ERR_INVALID_ARG, "NULL pointer or M < 1");
+  if (!aligned16(X) || !aligned16(codes) || !aligned16(scales) || !aligned16(T))
+    return fail(SVDQ_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  return launch_k1(h, X, M, static_cast<uint8_t*>(codes), scales, static_cast<__nv_bfloat16*>(T),
+                   static_cast<cudaStream_t>(stream));
+}
+
+svdq_status svdq_attach_lora(svdq_layer_t h, const void* A, const void* B, int r_l, float scale, void* stream) {
+  if (check_layer(h)) return SVDQ_ERR_INVALID_ARG;
+  if (!A || !B || r_l < 1) return fail(SVDQ_ERR_INVALID_ARG, "bad LoRA arguments");
+  if (h->rank + r_l > 256) return fail(SVDQ_ERR_INVALID_ARG, "rank + r_l exceeds 256");
+  if (!std::isfinite(scale)) return fail(SVDQ_ERR_INVALID_ARG, "scale must be finite");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int new_rank = h->rank + r_l;
+  const int RP_new = round_up(new_rank, 32);
+  __nv_bfloat16 *L1T = nullptr, *L2T = nullptr;
+  svdq_status e;
+  if ((e = dalloc(&L1T, static_cast<size_t>(RP_new) * h->K * 2))) return e;
+  if ((e = dalloc(&L2T, static_cast<size_t>(h->N_pad) * RP_new * 2))) return cudaFree(L1T), e;
+  if (launch_lora_concat(h->L1T, h->L2T, h->K, h->N, h->N_pad, h->rank, h->RP, h->s,
+                         static_cast<const __nv_bfloat16*>(A), static_cast<const __nv_bfloat16*>(B), r_l, scale, RP_new,
+                         L1T, L2T, st) != cudaSuccess) {
+    cudaFree(L1T);
+    cudaFree(L2T);
+    return fail(SVDQ_ERR_CUDA, "LoRA concat launch failed");
+  }
+  cudaError_t ce = cudaStreamSynchronize(st);
+  if (ce != cudaSuccess) {
+    cudaFree(L1T);
+    cudaFree(L2T);
+    return fail(SVDQ_ERR_CUDA, cudaGetErrorString(ce));
+  }
+  cudaFree(h->L1T);
+  cudaFree(h->L2T);
+  h->L1T = L1T;
+  h->L2T = L2T;
+  h->rank = new_rank;
+  h->RP = RP_new;
+  return build_static_maps(h);
+}
+
+svdq_status svdq_layer_get_info(svdq_layer_t h, svdq_layer_info* info) {
+  if (check_layer(h)) return SVDQ_ERR_INVALID_ARG;
+  if (!info) return fail(SVDQ_ERR_INVALID_ARG, "info is NULL");
+  info->K = h->K;
+  info->N = h->N;
+  info->rank = h->rank;
+  info->rank_pad = h->RP;
+  info->fmt = h->fmt;
+  info->alpha = h->cfg.alpha;
+  info->g_x = h->g_x;
+  info->g_w = h->g_w;
+  info->t_scale = h->t_scale;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_export_weights(svdq_layer_t h, void* blob, size_t* bytes, void* stream) {
+  if (check_layer(h)) return SVDQ_ERR_INVALID_ARG;
+  if (!bytes) return fail(SVDQ_ERR_INVALID_ARG, "bytes is NULL");
+  const int K = h->K, N = h->N, r = h->rank;
+  const bool i4 = h->fmt == SVDQ_INT4_G64;
+  svdq_blob_header hd{};
+  hd.magic = 0x51445653u;
+  hd.version = 1;
+  hd.fmt = h->fmt;
+  hd.K = K;
+  hd.N = N;
+  hd.rank = r;
+  hd.alpha = h->cfg.alpha;
+  hd.g_x = h->g_x;
+  hd.g_w = h->g_w;
+  size_t off = align256(sizeof(svdq_blob_header));
+  auto take = [&](size_t n) {
+    size_t o = off;
+    off = align256(off + n);
+    return static_cast<uint64_t>(o);
+  };
+  hd.off_s = take(K * 4);
+  hd.off_inv_s = take(K * 4);
+  hd.off_L1 = take(static_cast<size_t>(K) * r * 2);
+  hd.off_L2 = take(static_cast<size_t>(r) * N * 2);
+  hd.off_codes = take(static_cast<size_t>(N) * K / 2);
+  hd.off_scales = take(i4 ? static_cast<size_t>(N) * (K / 64) * 4 : static_cast<size_t>(N) * (K / 16));
+  hd.off_bias = take(N * 2);
+  hd.total = off;
+  if (!blob) {
+    *bytes = off;
+    return SVDQ_OK;
+  }
+  if (*bytes < off) return fail(SVDQ_ERR_INVALID_ARG, "blob too small");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* b = static_cast<uint8_t*>(blob);
+  std::memset(b, 0, off);
+  std::memcpy(b, &hd, sizeof(hd));
+  std::vector<uint16_t> l1t(static_cast<size_t>(h->RP) * K), l2t(static_cast<size_t>(h->N_pad) * h->RP);
+  const size_t cbytes = i4 ? static_cast<size_t>(h->N_pad) * K : static_cast<size_t>(h->N_pad) * K / 2;
+  const size_t sbytes = i4 ? static_cast<size_t>(K / 64) * h->N_pad * 4 : static_cast<size_t>(h->N_pad / 128) * (K / 64) * 512;
+  std::vector<uint8_t> codes(cbytes), scales(sbytes);
+  CUDA_TRY(cudaMemcpyAsync(b + hd.off_s, h->s, K * 4, cudaMemcpyDeviceToHost, st));
+  CUDA_TRY(cudaMemcpyAsync(b + hd.off_inv_s, h->inv_s, K * 4, cudaMemcpyDeviceToHost, st));
+  CUDA_TRY(cudaMemcpyAsync(b + hd.off_bias, h->bias, N * 2, cudaMemcpyDeviceToHost, st));
+  CUDA_TRY(cudaMemcpyAsync(l1t.data(), h->L1T, l1t.size() * 2, cudaMemcpyDeviceToHost, st));
+  CUDA_TRY(cudaMemcpyAsync(l2t.data(), h->L2T, l2t.size() * 2, cudaMemcpyDeviceToHost, st));
+  CUDA_TRY(cudaMemcpyAsync(codes.data(), h->wcodes, cbytes, cudaMemcpyDeviceToHost, st));
+  CUDA_TRY(cudaMemcpyAsync(scales.data(), h->wscales, sbytes, cudaMemcpyDeviceToHost, st));
+  CUDA_TRY(cudaStreamSynchronize(st));
+  uint16_t* L1 = reinterpret_cast<uint16_t*>(b + hd.off_L1);
+  uint16_t* L2 = reinterpret_cast<uint16_t*>(b + hd.off_L2);
+  for (int k = 0; k < K; ++k)
+    for (int j = 0; j < r; ++j) L1[static_cast<size_t>(k) * r + j] = l1t[static_cast<size_t>(j) * K + k];
+  for (int j = 0; j < r; ++j)
+    for (int n = 0; n < N; ++n) L2[static_cast<size_t>(j) * N + n] = l2t[static_cast<size_t>(n) * h->RP + j];
+  uint8_t* C = b + hd.off_codes;
+  if (i4) {
+    // E4M3 bytes of the integers -8..7 back to two's-complement nibbles
+    auto to_int = [](uint8_t e) -> int {
+      const int mag_code = e & 0x7F;
+      int mag = 0;
+      switch (mag_code) {
+        case 0x00: mag = 0; break;
+        case 0x38: mag = 1; break;
+        case 0x40: mag = 2; break;
+        case 0x44: mag = 3; break;
+        case 0x48: mag = 4; break;
+        case 0x4A: mag = 5; break;
+        case 0x4C: mag = 6; break;
+        case 0x4E: mag = 7; break;
+        case 0x50: mag = 8; break;
+        default: mag = 0; break;
+      }
+      return (e & 0x80) ? -mag : mag;
+    };
+    for (int n = 0; n < N; ++n)
+      for (int k = 0; k < K; k += 2) {
+        const int q0 = to_int(codes[static_cast<size_t>(n) * K + k]);
+        const int q1 = to_int(codes[static_cast<size_t>(n) * K + k + 1]);
+        C[static_cast<size_t>(n) * (K / 2) + k / 2] = static_cast<uint8_t>((q0 & 0xF) | ((q1 & 0xF) << 4));
+      }
+    float* S = reinterpret_cast<float*>(b + hd.off_scales);
+    const float* sw = reinterpret_cast<const float*>(scales.data());
+    for (int n = 0; n < N; ++n)
+      for (int g = 0; g < K / 64; ++g) S[static_cast<size_t>(n) * (K / 64) + g] = sw[static_cast<size_t>(g) * h->N_pad + n];
+  } else {
+    std::memcpy(C, codes.data(), static_cast<size_t>(N) * K / 2);
+    uint8_t* S = b + hd.off_scales;
+    for (int n = 0; n < N; ++n)
+      for (int i = 0; i < K / 16; ++i) {
+        const size_t atom = static_cast<size_t>(n / 128) * (K / 64) + i / 4;
+        S[static_cast<size_t>(n) * (K / 16) + i] = scales[atom * 512 + (n % 32) * 16 + ((n / 32) % 4) * 4 + i % 4];
+      }
+  }
+  *bytes = off;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_device_status(svdq_layer_t h, void* stream) {
+  if (check_layer(h)) return SVDQ_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  CUDA_TRY(cudaMemcpyAsync(&v, h->status, 4, cudaMemcpyDeviceToHost, st));
+  CUDA_TRY(cudaStreamSynchronize(st));
+  CUDA_TRY(cudaMemsetAsync(h->status, 0, 4, st));
+  if (v == kDevTimeout) return fail(SVDQ_ERR_DEVICE_TIMEOUT, "a kernel gave up a pipeline wait");
+  return SVDQ_OK;
+}
+
+svdq_status svdq_destroy(svdq_layer_t h) {
+  if (!h) return SVDQ_OK;
+  cudaDeviceSynchronize();
+  free_layer(h);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_selftest_bounded_wait(unsigned long long limit_ns, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* status = nullptr;
+  svdq_status e;
+  if ((e = dalloc(&status, 16))) return e;
+  int v = -1;
+  cudaError_t ce = cudaMemsetAsync(status, 0xFF, 4, st);
+  if (ce == cudaSuccess) ce = launch_wait_selftest(status, limit_ns, st);
+  if (ce == cudaSuccess) ce = cudaMemcpyAsync(&v, status, 4, cudaMemcpyDeviceToHost, st);
+  if (ce == cudaSuccess) ce = cudaStreamSynchronize(st);
+  cudaFree(status);
+  if (ce != cudaSuccess) return fail(SVDQ_ERR_CUDA, cudaGetErrorString(ce));
+  if (v == kDevTimeout) return fail(SVDQ_ERR_DEVICE_TIMEOUT, "bounded wait gave up as designed");
+  return SVDQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,164 @@
+"""CUDA path vs the oracle, element by element, through the C ABI (needs a B200).
+
+Stage by stage, each stage fed what the oracle fixes upstream:
+  prepare  (oracle SVD factors given)  s, inv_s, residual codes/scales, g_w, g_x: bit-exact
+  K1       activation codes and scales: bit-exact; T: normwise <= 2e-3
+  forward  Y: normwise <= 4e-3 against the oracle's float64 Y
+plus the full cuSOLVER prepare (factor product within 1e-5, Y within 4e-3),
+ragged shapes (M = 1, M and N off the tile grid, K off the NVFP4 k-tile), and
+the bounded-wait failure path.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import formats as F
+from oracle import svdquant as S
+from parity import T_TOL, Y_TOL, canonical_weight_codes, f64, gpu_activations, gpu_prepare, oracle_case, rel
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "cfg0_int4": lambda: workloads.config(0)[0],
+    "cfg0_nvfp4": lambda: _as_fmt(workloads.config(0)[0], workloads.NVFP4_G16),
+    "ragged_int4": lambda: workloads.custom(129, 384, 144, 40, workloads.INT4_G64, seed=71),
+    "ragged_nvfp4": lambda: workloads.custom(129, 384, 144, 40, workloads.NVFP4_G16, seed=72),
+    "m1_int4": lambda: workloads.custom(1, 256, 128, 8, workloads.INT4_G64, seed=73),
+    "m1_nvfp4": lambda: workloads.custom(1, 256, 128, 8, workloads.NVFP4_G16, seed=74),
+    "rank100_nvfp4": lambda: workloads.custom(300, 512, 256, 100, workloads.NVFP4_G16, seed=75),
+    "rank100_int4": lambda: workloads.custom(300, 512, 256, 100, workloads.INT4_G64, seed=76),
+}
+
+
+def _as_fmt(layer, fmt):
+    layer.fmt = fmt
+    layer.name += "_" + fmt
+    return layer
+
+
+@pytest.fixture(scope="module", params=sorted(SMALL))
+def small(request):
+    case = oracle_case(SMALL[request.param]())
+    g = gpu_prepare(case, with_factors=True)
+    yield case, g
+    g.close()
+
+
+def test_bounded_wait_gives_up_and_context_survives():
+    import rank_gemm_quantize_b200 as rq
+    st = rq.selftest_bounded_wait(50_000_000)
+    assert st == rq.Status.DEVICE_TIMEOUT
+    x = torch.arange(1024, device="cuda", dtype=torch.float32)
+    assert float(x.sum()) == 1023 * 1024 / 2
+
+
+def test_prepare_matches_oracle_bit_exact(small):
+    case, g = small
+    ex = g.export()
+    p = case.p
+    assert np.array_equal(ex["s"].view(np.uint32), p.s.view(np.uint32))
+    assert np.array_equal(ex["inv_s"].view(np.uint32), p.inv_s.view(np.uint32))
+    assert np.array_equal(ex["L1"], p.L1) and np.array_equal(ex["L2"], p.L2)
+    assert np.array_equal(ex["bias"], p.bias)
+    assert np.array_equal(ex["codes_packed"], canonical_weight_codes(p))
+    if p.fmt == workloads.INT4_G64:
+        assert np.array_equal(ex["scales"].view(np.uint32), p.w_scales.view(np.uint32))
+    else:
+        assert np.array_equal(ex["scales"], p.w_scales)
+        assert ex["g_w"] == p.g_w and ex["g_x"] == p.g_x
+
+
+def test_activation_kernel_matches_oracle(small):
+    case, g = small
+    L = case.layer
+    q, sc, T, pad_ok = gpu_activations(g, L.X.cuda(), L.fmt, L.M, L.K)
+    assert pad_ok
+    assert np.array_equal(q, case.r.x_codes), f"{np.sum(q != case.r.x_codes)} codes differ"
+    if L.fmt == workloads.INT4_G64:
+        assert np.array_equal(sc.view(np.uint32), case.r.x_scales.view(np.uint32))
+    else:
+        assert np.array_equal(sc, case.r.x_scales)
+    assert rel(T[:, :L.rank], case.r.T) <= T_TOL
+    assert np.all(T[:, L.rank:] == 0)
+
+
+def test_forward_matches_oracle(small):
+    case, g = small
+    L = case.layer
+    Y = g.forward(L.X.cuda())
+    torch.cuda.synchronize()
+    y = f64(Y)
+    assert np.all(np.isfinite(y))
+    err = rel(y, case.r.Y)
+    assert err <= Y_TOL, err
+    assert g.device_status() == 0
+
+
+def test_forward_is_deterministic_and_reuses_workspace(small):
+    case, g = small
+    X = case.layer.X.cuda()
+    y1 = g.forward(X).clone()
+    y2 = g.forward(X)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
+@pytest.mark.parametrize("name", ["cfg0_int4", "ragged_nvfp4", "rank100_int4"])
+def test_full_prepare_with_cusolver_svd(name):
+    case = oracle_case(SMALL[name]())
+    g = gpu_prepare(case, with_factors=False)
+    try:
+        ex = g.export()
+        assert np.array_equal(ex["s"].view(np.uint32), case.p.s.view(np.uint32))
+        prod_gpu = ex["L1"] @ ex["L2"]
+        prod_orc = case.p.L1 @ case.p.L2
+        assert rel(prod_gpu, prod_orc) <= 1e-5
+        Y = g.forward(case.layer.X.cuda())
+        torch.cuda.synchronize()
+        assert rel(f64(Y), case.r.Y) <= Y_TOL
+    finally:
+        g.close()
+
+
+@pytest.mark.parametrize("fmt", workloads.FORMATS)
+def test_lora_attach_leaves_residual_untouched(fmt):
+    layer = workloads.custom(192, 512, 256, 16, fmt, seed=81, lora_rank=32)
+    case = oracle_case(layer)
+    g = gpu_prepare(case)
+    try:
+        before = g.export()
+        g.attach_lora(layer.lora_A.cuda(), layer.lora_B.cuda(), 0.75)
+        after = g.export()
+        assert np.array_equal(before["codes_packed"], after["codes_packed"])
+        assert np.array_equal(before["scales"], after["scales"])
+        q = S.attach_lora(case.p, workloads.to_f64(layer.lora_A), workloads.to_f64(layer.lora_B), 0.75)
+        assert after["rank"] == 48
+        assert np.array_equal(after["L1"], q.L1) and np.array_equal(after["L2"], q.L2)
+        Y = g.forward(layer.X.cuda())
+        torch.cuda.synchronize()
+        yq = S.forward(q, case.X).Y
+        assert rel(f64(Y), yq) <= Y_TOL
+    finally:
+        g.close()
+
+
+def test_full_size_attention_projection_int4():
+    """The benchmark's workload (FLUX attention projection, 4608 x 3072 x 3072,
+    r 32, INT4 g64) in the same launch configuration, every output checked."""
+    case = oracle_case(workloads.config(1)[0])
+    g = gpu_prepare(case)
+    try:
+        ex = g.export()
+        assert np.array_equal(ex["codes_packed"], canonical_weight_codes(case.p))
+        L = case.layer
+        X = L.X.cuda()
+        q, sc, T, _ = gpu_activations(g, X, L.fmt, L.M, L.K)
+        assert np.array_equal(q, case.r.x_codes)
+        assert np.array_equal(sc.view(np.uint32), case.r.x_scales.view(np.uint32))
+        assert rel(T[:, :L.rank], case.r.T) <= T_TOL
+        Y = g.forward(X)
+        torch.cuda.synchronize()
+        assert rel(f64(Y), case.r.Y) <= Y_TOL
+    finally:
+        g.close()
