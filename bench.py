@@ -1,0 +1,500 @@
+#!/usr/bin/env python
+"""Benchmark of the SVDQuant W4A4 + low-rank linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 1]
+
+One step = one pass of the whole hot path (svdq_linear_forward: the activation
+kernel + the 4-bit GEMM with the fused low-rank/bias epilogue) over one batch
+of the configuration's synthetic inputs (for the MLP-pair configurations, both
+layers). Default workload: the FLUX-like attention projection (X [4608, 3072]
+bf16, W [3072, 3072], rank 32, INT4 group 64). Prints one JSON line on rank 0.
+
+Multi-GPU (torchrun, one process per GPU): the layer is token-parallel - every
+rank runs its own batch against its own copy of the weights, with no
+collective on the data path (weak scaling); only the timing uses a barrier and
+a max-reduce over ranks.
+
+--impl reference times the CPU oracle (oracle/, float64 numpy) on the host
+cores on a row sample of the same workload, sized so the run ends in minutes.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A4+low-rank linear TOPS & µs/layer (FLUX shapes), % of FP4/INT8 tensor peak"
+L2_BYTES = 126 * 2 ** 20
+# dense datasheet peaks (context): FP4 9.0 PFLOP/s, INT8/FP8 4.5 POPS
+DATASHEET_TOPS = {"nvfp4_g16": 9000.0, "int4_g64": 4500.0}
+# tensor-rate ratio of the MMA kind each format runs on, relative to bf16
+RATE_VS_BF16 = {"nvfp4_g16": 4.0, "int4_g64": 2.0}  # mxf4nvf4 = 4x bf16; f8f6f4 = 2x bf16
+
+# DRAM bytes per launch from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
+# valid only while the kernel source it was taken from is unchanged.
+TRAFFIC_RECORDS_FILE = os.path.join(ROOT, "profiles", "traffic_records.txt")
+
+
+def workload_desc(cfg: int, layers) -> str:
+    L = layers[0]
+    if cfg == 1:
+        return f"FLUX-like attention projection: X bf16 [{L.M},{L.K}] x W [{L.K},{L.N}], rank {L.rank}, {L.fmt}"
+    if cfg in (2, 3):
+        return (f"FLUX-like MLP pair: up [{L.M},{L.K}]x[{L.K},{L.N}] then down [{L.M},{layers[1].K}]x"
+                f"[{layers[1].K},{layers[1].N}], rank {L.rank}, {L.fmt}")
+    if cfg == 4:
+        return f"sweep point K=N=3072, M={L.M}, rank {L.rank}, {L.fmt}"
+    return f"single linear [{L.M},{L.K}]x[{L.K},{L.N}], rank {L.rank}, {L.fmt}"
+
+
+def layer_ops(M, K, N, r) -> float:
+    return 2.0 * M * K * N + 2.0 * M * r * (K + N)
+
+
+def gemm_ops(M, K, N, r) -> float:
+    return 2.0 * M * K * N + 2.0 * M * r * N
+
+
+def k1_bytes(M, K, r, fmt) -> float:
+    """Algorithmic HBM bytes of the activation kernel: X read, 4-bit codes and
+    group scales written, T written, L1 read once."""
+    G = 64 if fmt == "int4_g64" else 16
+    sbytes = 4 if fmt == "int4_g64" else 1
+    return 2.0 * M * K + M * K / 2 + M * K / G * sbytes + 2.0 * M * r + 2.0 * K * r
+
+
+def load_layers(args):
+    import workloads
+    kw = {}
+    if args.M:
+        kw["M"] = args.M
+    if args.rank:
+        kw["rank"] = args.rank
+    if args.fmt:
+        kw["fmt"] = args.fmt
+    layers = workloads.config(args.config, **kw)
+    return layers
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def source_digest(files) -> str:
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, workload_key: str):
+    """Per-launch DRAM bytes recorded from ncu, or None when absent or stale."""
+    if not os.path.exists(TRAFFIC_RECORDS_FILE):
+        return None
+    with open(TRAFFIC_RECORDS_FILE) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) < 5 or line.startswith("#"):
+                continue
+            name, wk, nbytes, digest, src = parts[0], parts[1], parts[2], parts[3], parts[4].split(",")
+            if name == kernel and wk == workload_key:
+                try:
+                    if source_digest(src) == digest:
+                        return float(nbytes)
+                except OSError:
+                    return None
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.25)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return {"samples": 0, "note": "nvidia-smi unavailable"}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        inside = [l for (t, l) in self.lines if t0 <= t <= t1 + 0.1]
+        use = inside or [l for (_, l) in self.lines]
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in use:
+            p = [x.strip() for x in l.split(",")]
+            if len(p) < 8:
+                continue
+            try:
+                sm.append(float(p[0]))
+                mx.append(float(p[1]))
+            except ValueError:
+                continue
+            for name, v in zip(names, p[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm), "samples_inside_timed_region": len(inside)}
+
+
+def init_dist(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    return world, rank, local
+
+
+def run_ours(args):
+    import datetime
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import rank_gemm_quantize_b200 as rq
+
+    world, rank, local = init_dist(args)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    layers = load_layers(args)
+    peaks, peak_kind = read_peaks()
+
+    # ---- prepare: one layer instance per rotating set (the first with the GPU
+    # SVD, the others from its factors), plus X / Y / workspace per set
+    preps = []
+    for L in layers:
+        X0 = L.X.to(dev)
+        a = rq.calibrate_absmax(X0)
+        g0 = rq.Layer.prepare(L.W.to(dev), L.bias.to(dev), a, L.fmt, L.rank, alpha=L.alpha)
+        ex = g0.export()
+        preps.append((L, X0, a, g0, ex))
+    set_bytes = 0
+    for (L, X0, a, g0, ex) in preps:
+        set_bytes += L.M * L.K * 2 + L.M * L.N * 2 + g0.workspace_size(L.M)
+        set_bytes += L.N * L.K // 2 * (2 if L.fmt == "int4_g64" else 1) + L.N * L.K // 16
+    n_sets = max(2, math.ceil(2 * L2_BYTES / max(set_bytes, 1)))
+    sets = []
+    for s in range(n_sets):
+        items = []
+        for (L, X0, a, g0, ex) in preps:
+            if s == 0:
+                g = g0
+            else:
+                L1 = torch.from_numpy(ex["L1"]).to(torch.bfloat16).to(dev)
+                L2 = torch.from_numpy(ex["L2"]).to(torch.bfloat16).to(dev)
+                g = rq.Layer.prepare(L.W.to(dev), L.bias.to(dev), a, L.fmt, L.rank, alpha=L.alpha, factors=(L1, L2))
+            X = X0 if s == 0 else X0.clone()
+            Y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(g.workspace_size(L.M), dtype=torch.uint8, device=dev)
+            items.append((g, X, Y, ws))
+        sets.append(items)
+    torch.cuda.synchronize()
+
+    n_layers = len(layers)
+    K_steps, W_steps = args.steps, args.warmup
+    # events: per step and layer, before K1 / between / after the GEMM
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_layers)] for _ in range(K_steps)]
+    for per_step in evs:  # torch creates the CUDA event at its first record
+        for per_layer in per_step:
+            for e in per_layer:
+                e.record()
+
+    def step(i, events=None):
+        for li, (g, X, Y, ws) in enumerate(sets[i % n_sets]):
+            if events is None:
+                g.forward(X, out=Y, workspace=ws)
+            else:
+                g.forward_profiled(X, Y, ws, events[li])
+
+    for i in range(W_steps):
+        step(i)
+    torch.cuda.synchronize()
+
+    uuid = str(torch.cuda.get_device_properties(local).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0_wall = time.time()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(K_steps):
+        step(i, evs[i])
+    end.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t1_wall = time.time()
+    clocks = sampler.stop(t0_wall, t1_wall)
+    elapsed_ms = start.elapsed_time(end)
+    k1_ms = [statistics.fmean(evs[i][li][0].elapsed_time(evs[i][li][1]) for i in range(K_steps)) for li in range(n_layers)]
+    gemm_ms = [statistics.fmean(evs[i][li][1].elapsed_time(evs[i][li][2]) for i in range(K_steps)) for li in range(n_layers)]
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+
+    step_ops = sum(layer_ops(L.M, L.K, L.N, L.rank) for L in layers)
+    value = step_ops * K_steps * world / (max_ms * 1e-3) / 1e12
+    ms_per_step = max_ms / K_steps
+
+    # ---- e2e through the public API with host buffers: H2D of X, forward, D2H of Y
+    e2e_steps = max(3, min(args.e2e_steps, K_steps))
+    hostX = [L.X.pin_memory() for L in layers]
+    hostY = [torch.empty(L.M, L.N, dtype=torch.bfloat16).pin_memory() for L in layers]
+    h2d = sum(L.M * L.K * 2 for L in layers)
+    d2h = sum(L.M * L.N * 2 for L in layers)
+
+    def e2e_step(i):
+        for li, (g, X, Y, ws) in enumerate(sets[i % n_sets]):
+            X.copy_(hostX[li], non_blocking=True)
+            g.forward(X, out=Y, workspace=ws)
+            hostY[li].copy_(Y, non_blocking=True)
+
+    for i in range(2):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = step_ops * e2e_steps * world / (float(te.item()) * 1e-3) / 1e12
+
+    # device status: no kernel gave up a wait
+    for items in sets:
+        for (g, X, Y, ws) in items:
+            if g.device_status() != rq.Status.OK:
+                raise SystemExit("a kernel reported a timed-out pipeline wait")
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    # ---- roofline of the dominant kernel (the GEMM) and of the activation kernel
+    fmt = layers[0].fmt
+    wl_key = f"cfg{args.config}_M{layers[0].M}_r{layers[0].rank}_{fmt}"
+    g_ops = sum(gemm_ops(L.M, L.K, L.N, L.rank) for L in layers)
+    g_s = sum(gemm_ms) * 1e-3
+    tensor_peak = peaks["bf16_tflops_sustained"] * RATE_VS_BF16[fmt]
+    gemm_name = "gemm_int4_kernel" if fmt == "int4_g64" else "gemm_nvfp4_kernel"
+    traffic = traffic_for(gemm_name, wl_key)
+    roofline = {"bound": "tensor", "kernel": gemm_name, "achieved": g_ops / g_s / 1e12,
+                "peak": tensor_peak, "unit": "TFLOP/s", "frac": g_ops / g_s / 1e12 / tensor_peak,
+                "traffic": traffic,
+                "peak_source": (f"{peak_kind} bf16 sustained {peaks['bf16_tflops_sustained']} TFLOP/s x "
+                                f"{RATE_VS_BF16[fmt]:g} (nominal {'mxf4nvf4' if fmt == 'nvfp4_g16' else 'f8f6f4'}/bf16 rate)"),
+                "algorithmic": "2MKN + 2MrN per launch", "frac_of_datasheet_dense": g_ops / g_s / 1e12 / DATASHEET_TOPS[fmt]}
+    k_bytes = sum(k1_bytes(L.M, L.K, L.rank, fmt) for L in layers)
+    k_s = sum(k1_ms) * 1e-3
+    k1_roof = {"bound": "hbm", "kernel": "act_quant_kernel", "achieved": k_bytes / k_s / 1e9, "peak": peaks["hbm_gbs"],
+               "unit": "GB/s", "frac": k_bytes / k_s / 1e9 / peaks["hbm_gbs"],
+               "traffic": traffic_for("act_quant_kernel", wl_key),
+               "algorithmic": "2MK + MK/2 + MK/G*scale + 2Mr + 2Kr bytes per launch"}
+
+    cpu = None
+    if not args.no_cpu_baseline:
+        cpu = cpu_baseline(layers, budget_s=args.cpu_seconds)
+
+    out = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "TOPS",
+        "n_gpus": world,
+        "steps": K_steps,
+        "warmup": W_steps,
+        "ms_per_step": ms_per_step,
+        "us_per_layer": ms_per_step * 1e3 / n_layers,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int4" if fmt == "int4_g64" else "nvfp4",
+        "data": "synthetic",
+        "config": {"workload": workload_desc(args.config, layers), "config_id": args.config,
+                   "M": layers[0].M, "K": layers[0].K, "N": layers[0].N, "rank": layers[0].rank, "format": fmt,
+                   "layers_per_step": n_layers,
+                   "l2": f"inputs larger than L2: {n_sets} rotating sets of prepared layer + X/Y/workspace "
+                         f"({n_sets * set_bytes / 2**20:.0f} MiB > 2 x 126 MiB L2)"},
+        "pct_of_datasheet_dense_peak": 100.0 * value / DATASHEET_TOPS[fmt],
+        "roofline": roofline,
+        "kernels": {"act_quant": {"ms": k1_ms, **k1_roof}, "gemm": {"ms": gemm_ms}},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps, "ms_per_step": float(te.item()) / e2e_steps},
+        "gpu_launches": 2 * n_layers * K_steps,
+        "clocks": clocks,
+        "impl": "ours",
+    }
+    print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def _blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def _oracle_prepare(layers):
+    import workloads
+    from oracle import svdquant as S
+    out = []
+    for L in layers:
+        X = workloads.to_f64(L.X)
+        a = S.calibrate_absmax(X)
+        p = S.prepare(workloads.to_f64(L.W), workloads.to_f64(L.bias), a, L.fmt, L.alpha, L.rank)
+        S.dequantized_weight(p)
+        out.append((L, X, p))
+    return out
+
+
+def cpu_baseline(layers, budget_s: float = 10.0, rows=None):
+    """The oracle's forward timed on the host cores on a row sample of the workload."""
+    from oracle import svdquant as S
+    preps = _oracle_prepare(layers)
+    M = layers[0].M
+    r = rows or M
+    t_total, n, ops = 0.0, 0, 0.0
+    while True:
+        t = time.perf_counter()
+        for (L, X, p) in preps:
+            S.forward(p, X[:r])
+        t_total += time.perf_counter() - t
+        n += 1
+        ops += sum(layer_ops(r, L.K, L.N, L.rank) for L in layers)
+        if t_total >= budget_s or n >= 50:
+            break
+    return {"value": ops / t_total / 1e12, "unit": "TOPS", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{n} oracle forward(s) of {r} of {M} rows per layer ({len(layers)} layer(s)), "
+                      f"{t_total:.1f} s; prepare (numpy SVD) excluded"}
+
+
+def run_reference(args):
+    world, rank, _ = init_dist(args)
+    if rank != 0:
+        return  # rank 0 alone runs the CPU reference; the others exit without work
+    layers = load_layers(args)
+    from oracle import svdquant as S
+    preps = _oracle_prepare(layers)
+    # size the row sample so that warmup + steps fit in ~2 minutes
+    t = time.perf_counter()
+    for (L, X, p) in preps:
+        S.forward(p, X[:64])
+    per_row = max((time.perf_counter() - t) / 64, 1e-6)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    rows = int(max(1, min(layers[0].M, budget / per_row)))
+    for _ in range(args.warmup):
+        for (L, X, p) in preps:
+            S.forward(p, X[:rows])
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        for (L, X, p) in preps:
+            S.forward(p, X[:rows])
+    dt = time.perf_counter() - t
+    ops = sum(layer_ops(rows, L.K, L.N, L.rank) for L in layers) * args.steps
+    value = ops / dt / 1e12
+    fmt = layers[0].fmt
+    cores = _blas_threads()
+    sample = f"{rows} of {layers[0].M} rows per step per layer"
+    out = {
+        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(args.config, layers), "config_id": args.config, "M": layers[0].M,
+                   "K": layers[0].K, "N": layers[0].N, "rank": layers[0].rank, "format": fmt,
+                   "layers_per_step": len(layers)},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--M", type=int, default=0)
+    ap.add_argument("--rank", type=int, default=0)
+    ap.add_argument("--fmt", choices=["int4_g64", "nvfp4_g16"], default=None)
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

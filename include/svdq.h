@@ -135,6 +135,12 @@ SVDQ_API svdq_status svdq_workspace_size(svdq_layer_t layer, int M, size_t* byte
 SVDQ_API svdq_status svdq_linear_forward(svdq_layer_t layer, const void* X, int M, void* Y, void* workspace,
                                 size_t workspace_bytes, void* stream);
 
+/* svdq_linear_forward with per-kernel timing: events[0..2] are cudaEvent_t the
+ * caller created; they are recorded on `stream` before the activation kernel,
+ * between the two kernels and after the GEMM. Same work, same launches. */
+SVDQ_API svdq_status svdq_linear_forward_profiled(svdq_layer_t layer, const void* X, int M, void* Y, void* workspace,
+                                                  size_t workspace_bytes, void* stream, void* const* events);
+
 /* Attaches a LoRA adapter Y += scale X A B to the low-rank branch without
  * re-quantizing R (abstract: off-the-shelf LoRAs without re-quantization).
  * The branch sees X diag(s)^-1, so L1' = [L1 | bf16(diag(s) A)] and

@@ -12,6 +12,7 @@ in bfloat16 ("high precision (such as FP16)", section 2.4).
 """
 from __future__ import annotations
 
+import dataclasses
 from dataclasses import dataclass, field
 from typing import Optional
 
@@ -186,6 +187,15 @@ def smooth_activations(X, inv_s) -> np.ndarray:
     return (np.asarray(X, dtype=F32) * np.asarray(inv_s, dtype=F32)[None, :]).astype(F32)
 
 
+def dequantized_weight(p: Prepared) -> np.ndarray:
+    """Q(R) as float64 values [N, K] (computed once per prepared layer)."""
+    cached = getattr(p, "_wq", None)
+    if cached is None or cached[0] is not p.w_codes:
+        cached = (p.w_codes, dequantize(p.w_codes, p.w_scales, p.fmt, p.g_w))
+        object.__setattr__(p, "_wq", cached)
+    return cached[1]
+
+
 @dataclass
 class ForwardResult:
     Y: np.ndarray  # float64 [M, N], not rounded
@@ -206,8 +216,7 @@ def forward(p: Prepared, X) -> ForwardResult:
     x_hat = smooth_activations(X, p.inv_s)
     x_codes, x_scales = quantize_rows(x_hat, p.fmt, p.g_x)
     xq = dequantize(x_codes, x_scales, p.fmt, p.g_x)
-    wq = dequantize(p.w_codes, p.w_scales, p.fmt, p.g_w)
-    main = xq @ wq.T
+    main = xq @ dequantized_weight(p).T
     T = x_hat.astype(np.float64) @ p.L1
     Y = main + T @ p.L2 + p.bias[None, :]
     return ForwardResult(Y, x_codes, x_scales, T, main)
@@ -231,8 +240,6 @@ def attach_lora(p: Prepared, A, B, scale: float) -> Prepared:
     B = np.asarray(B, dtype=np.float64)
     sA = bf16_round(p.s.astype(np.float64)[:, None] * A)
     sB = bf16_round(np.float64(F32(scale)) * B)
-    q = Prepared(**{**p.__dict__})
-    q.L1 = np.concatenate([p.L1, sA], axis=1)
-    q.L2 = np.concatenate([p.L2, sB], axis=0)
-    q.rank = q.L1.shape[1]
-    return q
+    L1 = np.concatenate([p.L1, sA], axis=1)
+    L2 = np.concatenate([p.L2, sB], axis=0)
+    return dataclasses.replace(p, L1=L1, L2=L2, rank=L1.shape[1])

@@ -70,6 +70,7 @@ SIGNATURES = {
     "svdq_prepare_weights_with_factors": [ctypes.POINTER(_Config), _VP, _VP, _VP, _VP, _VP, _VP, ctypes.POINTER(_VP)],
     "svdq_workspace_size": [_VP, _I, ctypes.POINTER(_SZ)],
     "svdq_linear_forward": [_VP, _VP, _I, _VP, _VP, _SZ, _VP],
+    "svdq_linear_forward_profiled": [_VP, _VP, _I, _VP, _VP, _SZ, _VP, ctypes.POINTER(_VP)],
     "svdq_attach_lora": [_VP, _VP, _VP, _I, _F, _VP],
     "svdq_quantize_activations": [_VP, _VP, _I, _VP, _VP, _VP, _VP],
     "svdq_export_weights": [_VP, _VP, ctypes.POINTER(_SZ), _VP],
@@ -199,6 +200,13 @@ class Layer:
         return out
 
     __call__ = forward
+
+    def forward_profiled(self, X: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor, events, stream=None):
+        """forward() recording three torch.cuda.Event objects around its two kernels."""
+        arr = (ctypes.c_void_p * 3)(*[e.cuda_event for e in events])
+        _check(lib().svdq_linear_forward_profiled(self._h, _ptr(X), X.shape[0], _ptr(out), _ptr(workspace),
+                                                  workspace.numel(), _stream(stream), arr))
+        return out
 
     def quantize_activations(self, X: torch.Tensor, stream=None):
         """(codes, scales, T) of the activation kernel in its documented layouts."""

@@ -475,8 +475,12 @@ svdq_status svdq_workspace_size(svdq_layer_t h, int M, size_t* bytes) {
   return SVDQ_OK;
 }
 
-svdq_status svdq_linear_forward(svdq_layer_t h, const void* X, int M, void* Y, void* workspace, size_t ws_bytes,
-                                void* stream) {
+}  // extern "C"
+
+namespace {
+
+svdq_status forward_impl(svdq_layer* h, const void* X, int M, void* Y, void* workspace, size_t ws_bytes,
+                         void* stream, void* const* events) {
   if (check_layer(h)) return SVDQ_ERR_INVALID_ARG;
   if (!X || !Y || !workspace || M < 1) return fail(SVDQ_ERR_INVALID_ARG, "NULL pointer or M < 1");
   if (!aligned16(X) || !aligned16(Y) || (reinterpret_cast<uintptr_t>(workspace) & 255))
@@ -488,8 +492,10 @@ svdq_status svdq_linear_forward(svdq_layer_t h, const void* X, int M, void* Y, v
   uint8_t* codes = base + w.codes;
   void* scales = base + w.scales;
   __nv_bfloat16* T = reinterpret_cast<__nv_bfloat16*>(base + w.T);
+  if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[0]), st));
   svdq_status e = launch_k1(h, X, M, codes, scales, T, st);
   if (e) return e;
+  if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[1]), st));
   if (h->ws_key != workspace || h->M_key != M) {
     const bool i4 = h->fmt == SVDQ_INT4_G64;
     const uint64_t row = i4 ? h->K : h->K / 2;
@@ -521,7 +527,23 @@ svdq_status svdq_linear_forward(svdq_layer_t h, const void* X, int M, void* Y, v
   maps.l2 = h->map_l2;
   cudaError_t ce = h->fmt == SVDQ_INT4_G64 ? launch_gemm_int4(p, maps, st) : launch_gemm_nvfp4(p, maps, st);
   if (ce != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("GEMM kernel: ") + cudaGetErrorString(ce));
+  if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[2]), st));
   return SVDQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+svdq_status svdq_linear_forward(svdq_layer_t h, const void* X, int M, void* Y, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  return forward_impl(h, X, M, Y, workspace, ws_bytes, stream, nullptr);
+}
+
+svdq_status svdq_linear_forward_profiled(svdq_layer_t h, const void* X, int M, void* Y, void* workspace,
+                                         size_t ws_bytes, void* stream, void* const* events) {
+  if (!events || !events[0] || !events[1] || !events[2]) return fail(SVDQ_ERR_INVALID_ARG, "three events needed");
+  return forward_impl(h, X, M, Y, workspace, ws_bytes, stream, events);
 }
 
 svdq_status svdq_quantize_activations(svdq_layer_t h, const void* X, int M, void* codes, void* scales, void* T,
