@@ -20,11 +20,14 @@ enum DeviceStatus : int {
   kDevTimeout = 1,
 };
 
-// Upper bound for any spin on an mbarrier, in nanoseconds of %globaltimer.
-// A healthy pipeline wait is microseconds; a wait this long means a producer
-// never arrived, and the kernel gives up, records kDevTimeout and unwinds.
-#ifndef SVDQ_WAIT_LIMIT_NS
-#define SVDQ_WAIT_LIMIT_NS 2000000000ull
+// Upper bound for any spin on an mbarrier, in SM clock cycles (about two
+// seconds at B200 clocks). A healthy pipeline wait is microseconds; a wait
+// this long means a producer never arrived, and the kernel gives up, records
+// kDevTimeout and unwinds. The per-SM cycle counter is used because it is
+// cheap to read; a global-timer read on every contended wait would sit on the
+// pipeline's critical path.
+#ifndef SVDQ_WAIT_LIMIT_CYCLES
+#define SVDQ_WAIT_LIMIT_CYCLES 4000000000ll
 #endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -90,12 +93,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
                                           int* status) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  const long long t0 = clock64();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(a, parity)) return true;
     if ((it & 63u) == 63u) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > SVDQ_WAIT_LIMIT_NS) {
+      if (clock64() - t0 > SVDQ_WAIT_LIMIT_CYCLES) {
         *abort_flag = 1;
         if (status) atomicExch(status, kDevTimeout);
         return false;

@@ -21,8 +21,14 @@ struct ActQuantParams {
   float g_x;               // NVFP4 activation tensor scale
   float denom;             // NVFP4: fp32(6 * g_x)
   float t_scale;           // 1 (INT4) or 1 / (g_x g_w) (NVFP4)
+  int* status;             // device status word (kDevTimeout on a given-up wait)
 };
-cudaError_t launch_act_quant(const ActQuantParams& p, int fmt, int rp, cudaStream_t stream);
+struct ActQuantMaps {
+  CUtensorMap x;    // X [M, K] bf16, box {64, 32}, 128-byte swizzle
+  CUtensorMap l1t;  // L1T [RP, K] bf16, box {64, RP}, 128-byte swizzle
+};
+int act_quant_box_rows();
+cudaError_t launch_act_quant(const ActQuantParams& p, const ActQuantMaps& maps, int fmt, int rp, cudaStream_t stream);
 
 // ---------------------------------------------------------------- GEMMs
 struct GemmParams {
@@ -41,6 +47,8 @@ struct GemmMaps {
   CUtensorMap t;   // T [M_pad, RP] bf16
   CUtensorMap l2;  // L2T [N_pad, RP] bf16
 };
+int gemm_nvfp4_bn();  // tile width (rows of the weight box) of each GEMM
+int gemm_int4_bn();
 cudaError_t launch_gemm_nvfp4(const GemmParams& p, const GemmMaps& maps, cudaStream_t stream);
 cudaError_t launch_gemm_int4(const GemmParams& p, const GemmMaps& maps, cudaStream_t stream);
 

@@ -61,7 +61,39 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
   return r == CUDA_SUCCESS;
 }
 
-constexpr int kGemmBN = 128;
+// Weight-side padding: every GEMM tile width divides it, so per-tile scale
+// copies never leave the buffers.
+constexpr int kNPad = 256;
+inline int gemm_bn(int fmt) { return fmt == SVDQ_INT4_G64 ? gemm_int4_bn() : gemm_nvfp4_bn(); }
+
+// Small cache of tensor maps keyed by (device pointer, rows): encoding a map
+// costs microseconds of host time, and callers usually cycle through a few
+// buffers.
+template <int N>
+struct MapCache {
+  struct Entry {
+    const void* key = nullptr;
+    int rows = -1;
+    CUtensorMap a{}, b{};
+  };
+  Entry e[N];
+  int next = 0;
+  Entry* find(const void* key, int rows) {
+    for (auto& x : e)
+      if (x.key == key && x.rows == rows) return &x;
+    return nullptr;
+  }
+  Entry* insert(const void* key, int rows) {
+    Entry* x = &e[next];
+    next = (next + 1) % N;
+    x->key = key;
+    x->rows = rows;
+    return x;
+  }
+  void clear() {
+    for (auto& x : e) x = Entry{};
+  }
+};
 
 struct WsLayout {
   int M_pad;
@@ -84,11 +116,9 @@ struct svdq_layer {
   uint8_t* wcodes = nullptr;     // INT4 [N_pad, K] E4M3 bytes; NVFP4 [N_pad, K/2]
   void* wscales = nullptr;       // INT4 float [K/64][N_pad]; NVFP4 atoms [N_pad/128][K/64][512]
   int* status = nullptr;         // device status word
-  CUtensorMap map_b{}, map_l2{};
-  // per-workspace maps, rebuilt when the workspace pointer or M changes
-  const void* ws_key = nullptr;
-  int M_key = -1;
-  CUtensorMap map_a{}, map_t{};
+  CUtensorMap map_b{}, map_l2{}, map_l1t{};
+  MapCache<8> ws_maps;  // (workspace, M) -> activation codes map (a), T map (b)
+  MapCache<8> x_maps;   // (X, M) -> X map (a)
 };
 
 namespace {
@@ -155,14 +185,17 @@ void free_layer(svdq_layer* h) {
 svdq_status build_static_maps(svdq_layer* h) {
   const bool i4 = h->fmt == SVDQ_INT4_G64;
   const uint64_t row = i4 ? h->K : h->K / 2;
-  if (!make_map(&h->map_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, row, h->N_pad, row, 128, kGemmBN,
+  if (!make_map(&h->map_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, row, h->N_pad, row, 128, gemm_bn(h->fmt),
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (weight codes) failed");
   if (!make_map(&h->map_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->L2T, h->RP, h->N_pad, static_cast<uint64_t>(h->RP) * 2,
-                32, kGemmBN, CU_TENSOR_MAP_SWIZZLE_64B))
+                32, gemm_bn(h->fmt), CU_TENSOR_MAP_SWIZZLE_64B))
     return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (L2) failed");
-  h->M_key = -1;
-  h->ws_key = nullptr;
+  if (!make_map(&h->map_l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->L1T, h->K, h->RP, static_cast<uint64_t>(h->K) * 2, 64,
+                h->RP, CU_TENSOR_MAP_SWIZZLE_128B))
+    return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (L1) failed");
+  h->ws_maps.clear();
+  h->x_maps.clear();
   return SVDQ_OK;
 }
 
@@ -271,7 +304,7 @@ svdq_status start_prepare(const svdq_config* cfg, const void* W, const void* bia
   h->cfg = *cfg;
   h->K = cfg->K;
   h->N = cfg->N;
-  h->N_pad = round_up(cfg->N, 128);
+  h->N_pad = round_up(cfg->N, kNPad);
   h->rank = cfg->rank;
   h->RP = round_up(cfg->rank, 32);
   h->fmt = cfg->fmt;
@@ -397,7 +430,20 @@ svdq_status launch_k1(svdq_layer* h, const void* X, int M, uint8_t* codes, void*
   p.g_x = h->g_x;
   p.denom = h->denom;
   p.t_scale = h->t_scale;
-  cudaError_t e = launch_act_quant(p, h->fmt, h->RP, st);
+  p.status = h->status;
+  ActQuantMaps maps;
+  auto* xe = h->x_maps.find(X, M);
+  if (!xe) {
+    xe = h->x_maps.insert(X, M);
+    if (!make_map(&xe->a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, h->K, M, static_cast<uint64_t>(h->K) * 2, 64,
+                  act_quant_box_rows(), CU_TENSOR_MAP_SWIZZLE_128B)) {
+      xe->key = nullptr;
+      return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (X) failed");
+    }
+  }
+  maps.x = xe->a;
+  maps.l1t = h->map_l1t;
+  cudaError_t e = launch_act_quant(p, maps, h->fmt, h->RP, st);
   if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("activation kernel: ") + cudaGetErrorString(e));
   return SVDQ_OK;
 }
@@ -496,16 +542,18 @@ svdq_status forward_impl(svdq_layer* h, const void* X, int M, void* Y, void* wor
   svdq_status e = launch_k1(h, X, M, codes, scales, T, st);
   if (e) return e;
   if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[1]), st));
-  if (h->ws_key != workspace || h->M_key != M) {
+  auto* we = h->ws_maps.find(workspace, M);
+  if (!we) {
+    we = h->ws_maps.insert(workspace, M);
     const bool i4 = h->fmt == SVDQ_INT4_G64;
     const uint64_t row = i4 ? h->K : h->K / 2;
-    if (!make_map(&h->map_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, row, w.M_pad, row, 128, 128,
+    if (!make_map(&we->a, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, row, w.M_pad, row, 128, 128,
                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&h->map_t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, h->RP, w.M_pad, static_cast<uint64_t>(h->RP) * 2, 32,
-                  128, CU_TENSOR_MAP_SWIZZLE_64B))
+        !make_map(&we->b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, h->RP, w.M_pad, static_cast<uint64_t>(h->RP) * 2, 32,
+                  128, CU_TENSOR_MAP_SWIZZLE_64B)) {
+      we->key = nullptr;
       return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (activations) failed");
-    h->ws_key = workspace;
-    h->M_key = M;
+    }
   }
   GemmParams p{};
   p.M = M;
@@ -521,9 +569,9 @@ svdq_status forward_impl(svdq_layer* h, const void* X, int M, void* Y, void* wor
   p.out_scale = h->gxgw;
   p.status = h->status;
   GemmMaps maps;
-  maps.a = h->map_a;
+  maps.a = we->a;
   maps.b = h->map_b;
-  maps.t = h->map_t;
+  maps.t = we->b;
   maps.l2 = h->map_l2;
   cudaError_t ce = h->fmt == SVDQ_INT4_G64 ? launch_gemm_int4(p, maps, st) : launch_gemm_nvfp4(p, maps, st);
   if (ce != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("GEMM kernel: ") + cudaGetErrorString(ce));
