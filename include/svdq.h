@@ -141,6 +141,22 @@ SVDQ_API svdq_status svdq_linear_forward(svdq_layer_t layer, const void* X, int 
 SVDQ_API svdq_status svdq_linear_forward_profiled(svdq_layer_t layer, const void* X, int M, void* Y, void* workspace,
                                                   size_t workspace_bytes, void* stream, void* const* events);
 
+/* svdq_linear_forward for callers that cannot allocate device memory: hosts
+ * whose device memory belongs to their own allocator and may not be grown
+ * behind its back, or latency-critical loops where an allocation may
+ * synchronize the device. The pages describe no such call; it exists for
+ * these callers only. The workspace is a fixed 16 MiB scratch array inside
+ * the library's device image (held by every GPU that loads the library until
+ * the process exits); the caller passes only X and Y. Nothing is allocated
+ * and nothing needs clearing: the first kernel overwrites every byte the
+ * second one reads. Layers whose workspace for M rows exceeds 16 MiB are
+ * refused with SVDQ_ERR_INVALID_ARG (svdq_workspace_size gives the need).
+ * The first call on a device looks up the array's device address (set-up, once
+ * per device, with that device current); make that first call before any
+ * stream capture. All calls on a device share the array: calls whose work
+ * overlaps on the GPU race, so issue them on one stream. */
+SVDQ_API svdq_status svdq_linear_forward_noalloc(svdq_layer_t layer, const void* X, int M, void* Y, void* stream);
+
 /* Attaches a LoRA adapter Y += scale X A B to the low-rank branch without
  * re-quantizing R (abstract: off-the-shelf LoRAs without re-quantization).
  * The branch sees X diag(s)^-1, so L1' = [L1 | bf16(diag(s) A)] and

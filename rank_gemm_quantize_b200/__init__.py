@@ -71,6 +71,7 @@ SIGNATURES = {
     "svdq_workspace_size": [_VP, _I, ctypes.POINTER(_SZ)],
     "svdq_linear_forward": [_VP, _VP, _I, _VP, _VP, _SZ, _VP],
     "svdq_linear_forward_profiled": [_VP, _VP, _I, _VP, _VP, _SZ, _VP, ctypes.POINTER(_VP)],
+    "svdq_linear_forward_noalloc": [_VP, _VP, _I, _VP, _VP],
     "svdq_attach_lora": [_VP, _VP, _VP, _I, _F, _VP],
     "svdq_quantize_activations": [_VP, _VP, _I, _VP, _VP, _VP, _VP],
     "svdq_export_weights": [_VP, _VP, ctypes.POINTER(_SZ), _VP],
@@ -200,6 +201,14 @@ class Layer:
         return out
 
     __call__ = forward
+
+    def forward_noalloc(self, X: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """forward() on the library's fixed scratch array (no workspace, no allocation by the library)."""
+        M = X.shape[0]
+        if out is None:
+            out = torch.empty(M, self.info().N, dtype=torch.bfloat16, device=X.device)
+        _check(lib().svdq_linear_forward_noalloc(self._h, _ptr(X), M, _ptr(out), _stream(stream)))
+        return out
 
     def forward_profiled(self, X: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor, events, stream=None):
         """forward() recording three torch.cuda.Event objects around its two kernels."""

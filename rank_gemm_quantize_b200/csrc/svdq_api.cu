@@ -24,6 +24,15 @@ svdq_status fail(svdq_status st, const std::string& msg) {
   return st;
 }
 
+}  // namespace
+
+namespace svdq {
+// Lets other translation units of the library report through svdq_last_error.
+void set_last_error(const std::string& msg) { g_last_error = msg; }
+}  // namespace svdq
+
+namespace {
+
 #define CUDA_TRY(expr)                                                                              \
   do {                                                                                              \
     cudaError_t e__ = (expr);                                                                       \
