@@ -34,7 +34,7 @@ cudaError_t launch_act_quant(const ActQuantParams& p, const ActQuantMaps& maps, 
 struct GemmParams {
   int M, N, K, RP;
   __nv_bfloat16* Y;            // [M, N]
-  const __nv_bfloat16* bias;   // [N]
+  const __nv_bfloat16* bias;   // [N_pad], zero beyond N
   const void* sa;              // activation scales (layout of ActQuantParams::scales)
   const void* sb;              // weight scales: INT4 float [K/64][N_pad]; NVFP4 atoms [N_pad/128][K/64][512]
   int M_pad, N_pad;

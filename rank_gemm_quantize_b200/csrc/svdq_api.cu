@@ -121,7 +121,7 @@ struct svdq_layer {
   float* inv_s = nullptr;
   __nv_bfloat16* L1T = nullptr;  // [RP, K]
   __nv_bfloat16* L2T = nullptr;  // [N_pad, RP]
-  __nv_bfloat16* bias = nullptr; // [N]
+  __nv_bfloat16* bias = nullptr; // [N_pad], zero beyond N
   uint8_t* wcodes = nullptr;     // INT4 [N_pad, K] E4M3 bytes; NVFP4 [N_pad, K/2]
   void* wscales = nullptr;       // INT4 float [K/64][N_pad]; NVFP4 atoms [N_pad/128][K/64][512]
   int* status = nullptr;         // device status word
@@ -322,14 +322,12 @@ svdq_status start_prepare(const svdq_config* cfg, const void* W, const void* bia
     free_layer(h);
     return s;
   };
-  if ((e = dalloc(&h->s, K * 4)) || (e = dalloc(&h->inv_s, K * 4)) || (e = dalloc(&h->bias, N * 2)) ||
+  if ((e = dalloc(&h->s, K * 4)) || (e = dalloc(&h->inv_s, K * 4)) || (e = dalloc(&h->bias, h->N_pad * 2)) ||
       (e = dalloc(&h->status, 16)))
     return bail(e);
   cudaMemsetAsync(h->status, 0, 16, st);
-  if (bias)
-    cudaMemcpyAsync(h->bias, bias, N * 2, cudaMemcpyDeviceToDevice, st);
-  else
-    cudaMemsetAsync(h->bias, 0, N * 2, st);
+  cudaMemsetAsync(h->bias, 0, h->N_pad * 2, st);  // padded with zeros to the weight padding
+  if (bias) cudaMemcpyAsync(h->bias, bias, N * 2, cudaMemcpyDeviceToDevice, st);
 
   float* wstat = nullptr;
   if ((e = dalloc(&wstat, K * 4))) return bail(e);
