@@ -9,17 +9,19 @@
 // This kernel reads every X element from HBM once and produces all three in
 // the same pass.
 //
-// Work split: a thread-block cluster of S CTAs owns 128 rows; CTA r of the
+// Work split: a thread-block cluster of S CTAs owns 64 rows; CTA r of the
 // cluster walks its 1/S share of K in 64-column chunks (S is chosen so the
-// grid covers the SMs once). Per chunk:
-//   * warp 16 (one thread) streams the X tile [128 x 64] and the L1^T slice
-//     [RP x 64] into a shared-memory ring with TMA (128-byte swizzle);
-//   * warps 0-15 (8 rows each) smooth, quantize, store codes and scales, and
+// grid covers the SMs once and every cluster is resident). Per chunk:
+//   * warp 17 (one thread) streams the X tile [64 x 64], the L1^T slice
+//     [RP x 64] and the inv_s slice into a shared-memory ring with TMA / bulk
+//     copies (128-byte swizzle);
+//   * warps 0-15 (4 rows each) smooth, quantize, store codes and scales, and
 //     write x_hat as a bf16 high part and a bf16 remainder straight into a
-//     tcgen05 K-major operand buffer;
-//   * the same thread of warp 16 then issues tcgen05 kind::f16 MMAs
+//     tcgen05 K-major operand buffer (128 rows: the MMA's M; rows 64-127 stay
+//     zero and their results are ignored);
+//   * one thread of warp 16 then issues tcgen05 kind::f16 MMAs
 //     (M = 128, N = RP, bf16 x bf16 -> fp32) of hi and lo against L1 into a
-//     TMEM accumulator, so T carries float32-level accuracy before its store.
+//     TMEM accumulator, so T's only sizable error is its final bf16 store.
 // At the end the S partial T tiles are reduced through distributed shared
 // memory in a fixed rank order (deterministic), scaled and stored as bf16.
 //
@@ -36,26 +38,34 @@ namespace svdq {
 
 namespace {
 
-constexpr int kRows = 128;     // rows per cluster (one tcgen05 M)
-constexpr int kQWarps = 16;    // quantizing warps, 8 rows each
-constexpr int kThreads = (kQWarps + 1) * 32;
+constexpr int kRows = 64;      // rows per cluster
+constexpr int kMmaM = 128;     // tcgen05 M; operand rows >= kRows are zero
+constexpr int kQWarps = 16;    // quantizing warps, 4 rows each
+constexpr int kMmaWarp = kQWarps;      // TMEM owner + MMA issuer
+constexpr int kProdWarp = kQWarps + 1; // TMA producer
+constexpr int kThreads = (kQWarps + 2) * 32;
+constexpr int kPair = 1;               // chunks each quantizing warp processes per iteration
 constexpr int kChunk = 64;     // columns per chunk (one 128-byte swizzle atom of bf16)
 constexpr int kRedCols = 64;   // columns per cluster-reduction pass
 
 template <int RP>
 struct K1Shape {
-  static constexpr int kStages = RP <= 64 ? 4 : (RP <= 128 ? 3 : 2);
+  static constexpr int kStages = RP <= 64 ? 4 : (RP <= 224 ? 3 : 2);
+  // x_hat operand buffers: phase A runs up to this many chunks ahead of the MMA
+  static constexpr int kABufs = RP <= 128 ? 4 : 3;
   static constexpr int kX = kRows * 128;             // X tile of a chunk (bf16, 64 cols)
   static constexpr int kL = RP * 128;                // L1^T slice of a chunk
   static constexpr int kS = 1024;                    // inv_s slice of a chunk (256 B used, 1 KB keeps alignment)
   static constexpr int kStage = kX + kL + kS;
-  static constexpr int kA = 2 * kRows * 128;         // hi + lo MMA operand of a chunk
+  static constexpr int kAHalf = kMmaM * 128;         // one operand (hi or lo) of a chunk
+  static constexpr int kA = 2 * kAHalf;              // hi + lo MMA operand of a chunk
   static constexpr int kAOff = kStages * kStage;
-  static constexpr int kRedOff = kAOff + 2 * kA;
+  static constexpr int kRedOff = kAOff + kABufs * kA;
   static constexpr int kRedW = RP < kRedCols ? RP : kRedCols;
   static constexpr int kRed = kRows * kRedW * 4;
   static constexpr int kBarOff = kRedOff + kRed;
   static constexpr int kTotal = kBarOff + 256 + 1024;
+  static_assert(kTotal <= 232448, "shared memory budget");
   static constexpr uint32_t kTmemCols = RP <= 32 ? 32 : (RP <= 64 ? 64 : (RP <= 128 ? 128 : 256));
 };
 
@@ -91,63 +101,91 @@ __device__ __forceinline__ float4 ld_peer_v4(uint32_t addr) {
 }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// Quantize 8 consecutive smoothed values of one row (this lane's share of a
-// group), store the codes, and the group scale from one lane per group.
-template <int FMT>
-__device__ __forceinline__ void quantize8(const float (&v)[8], const ActQuantParams& p, int row, int k, int cs) {
-  float amax = 0.f;
+// Quantize NP independent sets of 8 consecutive smoothed values (each one
+// lane's share of a group in a different row or chunk), stage by stage so the
+// NP dependency chains interleave; then store the codes and, from one lane per
+// group, the group scales.
+template <int FMT, int NP>
+__device__ __forceinline__ void quantize_passes(const float (&v)[NP][8], const ActQuantParams& p, const int (&row)[NP],
+                                                const int (&k)[NP], int cs) {
+  float amax[NP];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
+  for (int u = 0; u < NP; ++u) {
+    const float m01 = fmaxf(fabsf(v[u][0]), fabsf(v[u][1])), m23 = fmaxf(fabsf(v[u][2]), fabsf(v[u][3]));
+    const float m45 = fmaxf(fabsf(v[u][4]), fabsf(v[u][5])), m67 = fmaxf(fabsf(v[u][6]), fabsf(v[u][7]));
+    amax[u] = fmaxf(fmaxf(m01, m23), fmaxf(m45, m67));
+  }
   if (FMT == SVDQ_INT4_G64) {
     // group of 64 = the 8 lanes sharing (lane >> 3)
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-    float scale = 0.f;
-    uint32_t lo = 0, hi = 0;
-    if (amax > 0.f) {
-      scale = __fdiv_rn(amax, 7.0f);
-      const float inv = __fdiv_rn(7.0f, amax);
+#pragma unroll
+    for (int o = 1; o <= 4; o <<= 1)
+#pragma unroll
+      for (int u = 0; u < NP; ++u) amax[u] = fmaxf(amax[u], __shfl_xor_sync(0xffffffffu, amax[u], o));
+    float scale[NP], inv[NP];
+#pragma unroll
+    for (int u = 0; u < NP; ++u) {
+      const float safe = amax[u] > 0.f ? amax[u] : 1.f;
+      scale[u] = amax[u] > 0.f ? __fdiv_rn(safe, 7.0f) : 0.f;
+      inv[u] = __fdiv_rn(7.0f, safe);
+    }
+    uint32_t lo[NP], hi[NP];
+#pragma unroll
+    for (int u = 0; u < NP; ++u) {
       // |v| <= amax and inv <= (7 / amax)(1 + 2^-24), so |v * inv| rounds to at
       // most 7: rint already lands in [-7, 7] and the [-8, 7] clamp never acts.
+      // An all-zero group gives v = 0 and codes 0 with the placeholder inv.
+      // The rounding must see the float-rounded product: an add-based
+      // round-to-integer (adding and subtracting 1.5 * 2^23) gets fused with
+      // the multiply into one FMA by the code generator, which rounds the exact
+      // product instead and flips products that land exactly on a half.
       float q[8];
 #pragma unroll
       for (int j = 0; j < 8; j += 2) {
-        const float2 pr = __fmul2_rn(make_float2(v[j], v[j + 1]), make_float2(inv, inv));
+        const float2 pr = __fmul2_rn(make_float2(v[u][j], v[u][j + 1]), make_float2(inv[u], inv[u]));
         q[j] = rintf(pr.x);
         q[j + 1] = rintf(pr.y);
       }
-      lo = cvt_e4m3x2(q[0], q[1]) | (cvt_e4m3x2(q[2], q[3]) << 16);
-      hi = cvt_e4m3x2(q[4], q[5]) | (cvt_e4m3x2(q[6], q[7]) << 16);
+      lo[u] = cvt_e4m3x2(q[0], q[1]) | (cvt_e4m3x2(q[2], q[3]) << 16);
+      hi[u] = cvt_e4m3x2(q[4], q[5]) | (cvt_e4m3x2(q[6], q[7]) << 16);
     }
-    uint8_t* dst = p.codes + static_cast<size_t>(row) * p.K + k;
-    *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
-    if (cs == 0) reinterpret_cast<float*>(p.scales)[static_cast<size_t>(k >> 6) * p.M_pad + row] = scale;
+#pragma unroll
+    for (int u = 0; u < NP; ++u) {
+      *reinterpret_cast<uint2*>(p.codes + static_cast<size_t>(row[u]) * p.K + k[u]) = make_uint2(lo[u], hi[u]);
+      if (cs == 0) reinterpret_cast<float*>(p.scales)[static_cast<size_t>(k[u] >> 6) * p.M_pad + row[u]] = scale[u];
+    }
   } else {
     // group of 16 = this lane and its neighbour (lane ^ 1)
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    const float r = __fdiv_rn(amax, p.denom);
-    const uint32_t sb = cvt_e4m3x2(r, 0.f) & 0xFFu;
-    const float eff = __fmul_rn(e4m3_to_float(sb), p.g_x);
-    uint32_t codes = 0;
-    if (eff != 0.f) {
-      const float inv = __frcp_rn(eff);
+#pragma unroll
+    for (int u = 0; u < NP; ++u) amax[u] = fmaxf(amax[u], __shfl_xor_sync(0xffffffffu, amax[u], 1));
+    uint32_t sb[NP];
+    float eff[NP];
+#pragma unroll
+    for (int u = 0; u < NP; ++u) {
+      sb[u] = cvt_e4m3x2(__fdiv_rn(amax[u], p.denom), 0.f) & 0xFFu;
+      eff[u] = __fmul_rn(e4m3_to_float(sb[u]), p.g_x);
+    }
+    uint32_t codes[NP];
+#pragma unroll
+    for (int u = 0; u < NP; ++u) {
+      const float inv = __frcp_rn(eff[u] != 0.f ? eff[u] : 1.f);
       float q[8];
 #pragma unroll
       for (int j = 0; j < 8; j += 2) {
-        const float2 pr = __fmul2_rn(make_float2(v[j], v[j + 1]), make_float2(inv, inv));
+        const float2 pr = __fmul2_rn(make_float2(v[u][j], v[u][j + 1]), make_float2(inv, inv));
         q[j] = pr.x;
         q[j + 1] = pr.y;
       }
-      codes = cvt_e2m1x8(q);
+      codes[u] = eff[u] != 0.f ? cvt_e2m1x8(q) : 0u;
     }
-    uint8_t* dst = p.codes + static_cast<size_t>(row) * (p.K >> 1) + (k >> 1);
-    *reinterpret_cast<uint32_t*>(dst) = codes;
-    if ((cs & 1) == 0) {
-      const int sf = k >> 4;  // scale index along the row
-      const size_t atom = static_cast<size_t>(row >> 7) * (p.K >> 6) + (sf >> 2);
-      const int off = (row & 31) * 16 + ((row >> 5) & 3) * 4 + (sf & 3);
-      reinterpret_cast<uint8_t*>(p.scales)[atom * 512 + off] = static_cast<uint8_t>(sb);
+#pragma unroll
+    for (int u = 0; u < NP; ++u) {
+      *reinterpret_cast<uint32_t*>(p.codes + static_cast<size_t>(row[u]) * (p.K >> 1) + (k[u] >> 1)) = codes[u];
+      if ((cs & 1) == 0) {
+        const int sf = k[u] >> 4;  // scale index along the row
+        const size_t atom = static_cast<size_t>(row[u] >> 7) * (p.K >> 6) + (sf >> 2);
+        const int off = (row[u] & 31) * 16 + ((row[u] >> 5) & 3) * 4 + (sf & 3);
+        reinterpret_cast<uint8_t*>(p.scales)[atom * 512 + off] = static_cast<uint8_t>(sb[u]);
+      }
     }
   }
 }
@@ -161,9 +199,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);  // [kStages] TMA landed
   uint64_t* empty = full + S::kStages;                             // [kStages] MMA done with the stage
-  uint64_t* aready = empty + S::kStages;                           // [2] operand written by warps 0-7
-  uint64_t* afree = aready + 2;                                    // [2] MMA done reading the operand
-  uint64_t* mma_done = afree + 2;
+  uint64_t* aready = empty + S::kStages;                           // [S::kABufs] operand written by warps 0-15
+  uint64_t* afree = aready + S::kABufs;                               // [S::kABufs] MMA done reading the operand
+  uint64_t* mma_done = afree + S::kABufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -182,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < S::kABufs; ++b) {
       mbar_init(&aready[b], kQWarps);
       mbar_init(&afree[b], 1);
     }
@@ -190,47 +228,59 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == kQWarps) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, S::kTmemCols);
     tmem_relinquish();
+  }
+  {
+    // operand rows kRows..kMmaM-1 are never written per chunk: clear them once
+    uint4* a = reinterpret_cast<uint4*>(smem + S::kAOff);
+    const int per_half = (kMmaM - kRows) * 128 / 16;
+    for (int i = threadIdx.x; i < 2 * S::kABufs * per_half; i += kThreads) {
+      const int half = i / per_half;  // (buffer, hi/lo)
+      a[(half * S::kAHalf + kRows * 128) / 16 + (i % per_half)] = make_uint4(0, 0, 0, 0);
+    }
+    fence_async_smem();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kQWarps) {
-    // ------------------------------------------------ TMA producer + MMA issuer
+  if (warp == kProdWarp) {
+    // ------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tensormap(&maps.x);
       prefetch_tensormap(&maps.l1t);
-      const uint32_t idesc = idesc_dense(kFmtF32, kFmtBF16, kFmtBF16, kRows, RP);
-      int issued = 0;
-      bool ok = true;
-      auto issue = [&](int j) -> bool {
+      int j = 0;
+      for (; j < nlocal; ++j) {
         const int s = j % S::kStages;
-        if (!mbar_wait(&empty[s], ((j / S::kStages) & 1) ^ 1, abort_flag, p.status)) return false;
+        if (!mbar_wait(&empty[s], ((j / S::kStages) & 1) ^ 1, abort_flag, p.status)) break;
         uint8_t* st = smem + s * S::kStage;
         mbar_arrive_expect_tx(&full[s], S::kX + S::kL + kChunk * 4);
         tma_load_2d(st, &maps.x, &full[s], (c_begin + j) * kChunk, m0);
         tma_load_2d(st + S::kX, &maps.l1t, &full[s], (c_begin + j) * kChunk, 0);
         bulk_load(st + S::kX + S::kL, p.inv_s + (c_begin + j) * kChunk, kChunk * 4, &full[s]);
-        return true;
-      };
-      for (; issued < nlocal && issued < S::kStages - 1 && ok; ++issued) ok = issue(issued);
-      for (int j = 0; j < nlocal && ok; ++j) {
-        if (issued < nlocal) {
-          ok = issue(issued);
-          if (!ok) break;
-          ++issued;
-        }
-        const int b = j & 1;
-        ok = mbar_wait(&aready[b], (j >> 1) & 1, abort_flag, p.status);
-        if (!ok) break;
+      }
+      if (j < nlocal) {
+        // gave up: let the copies still in flight land before the CTA exits
+        volatile int no_abort = 0;
+        for (int i = max(0, j - S::kStages); i < j; ++i)
+          mbar_wait(&full[i % S::kStages], (i / S::kStages) & 1, &no_abort, nullptr);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_dense(kFmtF32, kFmtBF16, kFmtBF16, kMmaM, RP);
+      for (int j = 0; j < nlocal; ++j) {
+        const int b = j % S::kABufs;
+        if (!mbar_wait(&aready[b], (j / S::kABufs) & 1, abort_flag, p.status)) break;
         tc_fence_after();
         const int s = j % S::kStages;
         const uint32_t a_hi = smem_u32(smem + S::kAOff + b * S::kA);
-        const uint32_t a_lo = a_hi + kRows * 128;
+        const uint32_t a_lo = a_hi + S::kAHalf;
         const uint32_t bt = smem_u32(smem + s * S::kStage + S::kX);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
@@ -241,12 +291,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit(&empty[s]);
         tc_commit(&afree[b]);
       }
-      if (!ok) {
-        // let the copies still in flight land before the CTA exits
-        volatile int no_abort = 0;
-        for (int j = max(0, issued - S::kStages); j < issued; ++j)
-          mbar_wait(&full[j % S::kStages], (j / S::kStages) & 1, &no_abort, nullptr);
-      }
       tc_commit(mma_done);  // arrives once every MMA issued above has finished
     }
     __syncwarp();
@@ -255,51 +299,86 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int cs = lane & 7;   // 16-byte column segment of the chunk
     const int rl = lane >> 3;  // row within a 4-row pass
     const int r0 = warp * (kRows / kQWarps);  // this warp's rows
-    for (int j = 0; j < nlocal; ++j) {
-      const int s = j % S::kStages;
-      const int b = j & 1;
-      if (!mbar_wait(&full[s], (j / S::kStages) & 1, abort_flag, p.status)) break;
-      if (j >= 2 && !mbar_wait(&afree[b], ((j >> 1) & 1) ^ 1, abort_flag, p.status)) break;
-      const uint8_t* xt = smem + s * S::kStage;
-      uint8_t* ahi = smem + S::kAOff + b * S::kA;
-      uint8_t* alo = ahi + kRows * 128;
-      const int k = (c_begin + j) * kChunk + cs * 8;
-      const float* inv_s = reinterpret_cast<const float*>(xt + S::kX + S::kL) + cs * 8;
-      const float4 is0 = *reinterpret_cast<const float4*>(inv_s);
-      const float4 is1 = *reinterpret_cast<const float4*>(inv_s + 4);
-      const float is[8] = {is0.x, is0.y, is0.z, is0.w, is1.x, is1.y, is1.z, is1.w};
+    bool ok = true;
+    for (int j0 = 0; j0 < nlocal && ok; j0 += kPair) {
+      const int npair = min(kPair, nlocal - j0);
+      for (int u = 0; u < npair && ok; ++u) {
+        const int j = j0 + u;
+        ok = mbar_wait(&full[j % S::kStages], (j / S::kStages) & 1, abort_flag, p.status);
+        if (ok && j >= S::kABufs)
+          ok = mbar_wait(&afree[j % S::kABufs], ((j / S::kABufs) & 1) ^ 1, abort_flag, p.status);
+      }
+      if (!ok) break;
+      // The passes of the pair (and of the rows of this warp) are independent:
+      // every stage below runs over all of them, so their chains interleave.
+      constexpr int kPasses = kRows / kQWarps / 4;  // 4-row passes per chunk
+      constexpr int NP = kPair * kPasses;
+      float v[NP][8];
+      int rows[NP], ks[NP];
+      uint8_t* adst[NP];
+      int phys[NP];
 #pragma unroll
-      for (int i = 0; i < kRows / kQWarps / 4; ++i) {
-        const int lrow = r0 + 4 * i + rl;
-        const int phys = (cs ^ (lrow & 7)) * 16;
-        const uint4 xv = *reinterpret_cast<const uint4*>(xt + lrow * 128 + phys);
-        const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
-        float v[8];
+      for (int u = 0; u < kPair; ++u) {
+        const int j = j0 + (u < npair ? u : 0);  // a missing second chunk repeats the first (results unused)
+        const uint8_t* xt = smem + (j % S::kStages) * S::kStage;
+        const float* inv_s = reinterpret_cast<const float*>(xt + S::kX + S::kL) + cs * 8;
+        const float4 is0 = *reinterpret_cast<const float4*>(inv_s);
+        const float4 is1 = *reinterpret_cast<const float4*>(inv_s + 4);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          // one IEEE round-to-nearest product per element (packed pair)
-          const float2 pr = __fmul2_rn(make_float2(bf16_lo(w[e]), bf16_hi(w[e])), make_float2(is[2 * e], is[2 * e + 1]));
-          v[2 * e] = pr.x;
-          v[2 * e + 1] = pr.y;
+        for (int i = 0; i < kPasses; ++i) {
+          const int n = u * kPasses + i;
+          const int lrow = r0 + 4 * i + rl;
+          phys[n] = lrow * 128 + (cs ^ (lrow & 7)) * 16;
+          rows[n] = m0 + lrow;
+          ks[n] = (c_begin + j) * kChunk + cs * 8;
+          adst[n] = smem + S::kAOff + (j % S::kABufs) * S::kA;
+          const uint4 xv = *reinterpret_cast<const uint4*>(xt + phys[n]);
+          const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
+          const float is[8] = {is0.x, is0.y, is0.z, is0.w, is1.x, is1.y, is1.z, is1.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            // one IEEE round-to-nearest product per element (packed pair)
+            const float2 pr = __fmul2_rn(make_float2(bf16_lo(w[e]), bf16_hi(w[e])), make_float2(is[2 * e], is[2 * e + 1]));
+            v[n][2 * e] = pr.x;
+            v[n][2 * e + 1] = pr.y;
+          }
         }
-        quantize8<FMT>(v, p, m0 + lrow, k, cs);
-        uint32_t h[4], l[4];
+      }
+      if (npair == kPair) {
+        quantize_passes<FMT, NP>(v, p, rows, ks, cs);
+      } else {
+        float v1[kPasses][8];
+        int rows1[kPasses], ks1[kPasses];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * e]);
-          const __nv_bfloat16 h1 = __float2bfloat16_rn(v[2 * e + 1]);
-          const float d0 = v[2 * e] - __bfloat162float(h0);
-          const float d1 = v[2 * e + 1] - __bfloat162float(h1);
-          h[e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
-          l[e] = pack_bf16x2(d0, d1);
+        for (int n = 0; n < kPasses; ++n) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v1[n][e] = v[n][e];
+          rows1[n] = rows[n];
+          ks1[n] = ks[n];
         }
-        // same 128-byte swizzle as the TMA tiles: the canonical tcgen05 K-major layout
-        *reinterpret_cast<uint4*>(ahi + lrow * 128 + phys) = make_uint4(h[0], h[1], h[2], h[3]);
-        *reinterpret_cast<uint4*>(alo + lrow * 128 + phys) = make_uint4(l[0], l[1], l[2], l[3]);
+        quantize_passes<FMT, kPasses>(v1, p, rows1, ks1, cs);
+      }
+#pragma unroll
+      for (int n = 0; n < NP; ++n) {
+        if (n < npair * kPasses) {
+          uint32_t h[4], l[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            h[e] = pack_bf16x2(v[n][2 * e], v[n][2 * e + 1]);  // high parts, one packed conversion
+            // the remainders are exact in float: v - bf16(v) has at most 16 significant bits
+            const float2 d = __fadd2_rn(make_float2(v[n][2 * e], v[n][2 * e + 1]),
+                                        make_float2(-bf16_lo(h[e]), -bf16_hi(h[e])));
+            l[e] = pack_bf16x2(d.x, d.y);
+          }
+          // same 128-byte swizzle as the TMA tiles: the canonical tcgen05 K-major layout
+          *reinterpret_cast<uint4*>(adst[n] + phys[n]) = make_uint4(h[0], h[1], h[2], h[3]);
+          *reinterpret_cast<uint4*>(adst[n] + S::kAHalf + phys[n]) = make_uint4(l[0], l[1], l[2], l[3]);
+        }
       }
       fence_async_smem();  // make the generic-proxy writes visible to the tensor core
       __syncwarp();
-      if (lane == 0) mbar_arrive(&aready[b]);
+      if (lane == 0)
+        for (int u = 0; u < npair; ++u) mbar_arrive(&aready[(j0 + u) % S::kABufs]);
     }
   }
 
@@ -317,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp < 8 && healthy) {
       const int q = warp & 3;
       const int half = warp >> 2;
-      if (half * 32 < S::kRedW) {
+      if (half * 32 < S::kRedW && q * 32 < kRows) {
         uint32_t r[32];
         tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + c0 + half * 32, r);
         tmem_ld_wait();
@@ -362,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == kQWarps) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, S::kTmemCols);
   }

@@ -143,10 +143,22 @@ def test_lora_attach_leaves_residual_untouched(fmt):
         g.close()
 
 
-def test_full_size_attention_projection_int4():
-    """The benchmark's workload (FLUX attention projection, 4608 x 3072 x 3072,
-    r 32, INT4 g64) in the same launch configuration, every output checked."""
-    case = oracle_case(workloads.config(1)[0])
+def _half_ties_off_exact(case) -> int:
+    """How many INT4 activation products of this input round, in float32, to
+    exactly a half while the exact product does not: the elements that tell a
+    kernel which rounds the float32 product (as specified) from one that fuses
+    the multiply into its round-to-integer and rounds the exact product."""
+    xs = S.smooth_activations(case.X, case.p.inv_s)
+    g = xs.reshape(xs.shape[0], -1, 64)
+    amax = np.max(np.abs(g), axis=-1, keepdims=True)
+    inv = (np.float32(7.0) / np.where(amax == 0, np.float32(1.0), amax)).astype(np.float32)
+    prod = (g * inv).astype(np.float32)
+    tie = (prod - np.floor(prod)) == np.float32(0.5)
+    off = g.astype(np.float64) * inv.astype(np.float64) != prod.astype(np.float64)
+    return int(np.count_nonzero(tie & off))
+
+
+def _check_full_size(case):
     g = gpu_prepare(case)
     try:
         ex = g.export()
@@ -155,10 +167,33 @@ def test_full_size_attention_projection_int4():
         X = L.X.cuda()
         q, sc, T, _ = gpu_activations(g, X, L.fmt, L.M, L.K)
         assert np.array_equal(q, case.r.x_codes)
-        assert np.array_equal(sc.view(np.uint32), case.r.x_scales.view(np.uint32))
+        if L.fmt == workloads.INT4_G64:
+            assert np.array_equal(sc.view(np.uint32), case.r.x_scales.view(np.uint32))
+        else:
+            assert np.array_equal(sc, case.r.x_scales)
         assert rel(T[:, :L.rank], case.r.T) <= T_TOL
         Y = g.forward(X)
         torch.cuda.synchronize()
         assert rel(f64(Y), case.r.Y) <= Y_TOL
+        assert g.device_status() == 0
     finally:
         g.close()
+
+
+def test_full_size_attention_projection_int4():
+    """The benchmark's workload (FLUX attention projection, 4608 x 3072 x 3072,
+    r 32, INT4 g64) in the same launch configuration, every output checked.
+    Its activations hold products that land on exact halves only after float32
+    rounding; the test asserts they are there."""
+    case = oracle_case(workloads.config(1)[0])
+    assert _half_ties_off_exact(case) >= 5
+    _check_full_size(case)
+
+
+@pytest.mark.parametrize("cfg,which", [(2, 0), (2, 1), (3, 0), (3, 1)])
+def test_full_size_mlp_pair(cfg, which):
+    """The FLUX MLP pair at full size, every output checked: up 4608 x 3072 ->
+    12288 and down 4608 x 12288 -> 3072 (GELU of the up output, with outlier
+    channels), r 32, INT4 g64 (the first pair) and NVFP4 g16 (the second)."""
+    case = oracle_case(workloads.config(cfg)[which])
+    _check_full_size(case)
