@@ -182,6 +182,24 @@ class ClockSampler:
                 "samples": len(sm), "samples_inside_timed_region": len(inside)}
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's duration: the whole job is done when the last rank is."""
+    if world == 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tops(ops_per_rank_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Weak scaling: every rank runs its own batch of tokens through the layers
+    each step, so the job's work is world x the per-rank work, done in the
+    slowest rank's time."""
+    return ops_per_rank_step * steps * world / (max_ms * 1e-3) / 1e12
+
+
 def init_dist(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -280,13 +298,10 @@ def run_ours(args):
     elapsed_ms = start.elapsed_time(end)
     k1_ms = [statistics.fmean(evs[i][li][0].elapsed_time(evs[i][li][1]) for i in range(K_steps)) for li in range(n_layers)]
     gemm_ms = [statistics.fmean(evs[i][li][1].elapsed_time(evs[i][li][2]) for i in range(K_steps)) for li in range(n_layers)]
-    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = max_over_ranks(elapsed_ms, world, dev)
 
     step_ops = sum(layer_ops(L.M, L.K, L.N, L.rank) for L in layers)
-    value = step_ops * K_steps * world / (max_ms * 1e-3) / 1e12
+    value = whole_job_tops(step_ops, K_steps, world, max_ms)
     ms_per_step = max_ms / K_steps
 
     # ---- e2e through the public API with host buffers: H2D of X, forward, D2H of Y
@@ -313,10 +328,8 @@ def run_ours(args):
         e2e_step(i)
     e1.record()
     torch.cuda.synchronize()
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = step_ops * e2e_steps * world / (float(te.item()) * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = whole_job_tops(step_ops, e2e_steps, world, e2e_ms)
 
     # device status: no kernel gave up a wait
     for items in sets:
@@ -378,7 +391,7 @@ def run_ours(args):
         "kernels": {"act_quant": {"ms": k1_ms, **k1_roof}, "gemm": {"ms": gemm_ms}},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": e2e_steps, "ms_per_step": float(te.item()) / e2e_steps},
+                "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps},
         "gpu_launches": 2 * n_layers * K_steps,
         "clocks": clocks,
         "impl": "ours",
