@@ -56,11 +56,14 @@ struct SmemNv {
 };
 static_assert(SmemNv::kTotal <= 232448, "shared memory budget");
 
-// TMEM columns: accumulator [0, 256), A scale factors [256, 272), B scale
-// factors [272, 304).
+// TMEM columns: accumulator [0, 256), then one scale-factor slot per
+// shared-memory stage (A: 16 columns, B: 32), so copying the next k-tile's
+// scale factors never waits for the MMAs still reading the previous ones.
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSfSlotCols = 16 + 2 * 16;
 constexpr uint32_t kSfaCol = kBN;
 constexpr uint32_t kSfbCol = kBN + 16;
+static_assert(kBN + kStages * kSfSlotCols <= kTmemCols, "TMEM budget");
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_nvfp4_kernel(const GemmParams p, const __grid_constant__ GemmMaps maps) {
@@ -169,8 +172,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     const uint32_t idesc_main = idesc_block_scaled(kBM, kBN);
     const uint32_t idesc_lr = idesc_dense(kFmtF32, kFmtBF16, kFmtBF16, kBM, kBN);
-    const uint32_t t_sfa = tmem + kSfaCol;
-    const uint32_t t_sfb = tmem + kSfbCol;
     bool ok = true;
     int it = 0, ti = 0;
     for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++ti) {
@@ -189,6 +190,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b_base = smem_u32(st + L::kA);
           if (k < n_main) {
             const int nkb = min(4, kb_total - k * 4);
+            const uint32_t t_sfa = tmem + kSfaCol + s * kSfSlotCols;
+            const uint32_t t_sfb = tmem + kSfbCol + s * kSfSlotCols;
             const uint32_t sfa_base = smem_u32(st + L::kA + L::kB);
             const uint32_t sfb_base = sfa_base + L::kSfa;
             for (int j = 0; j < nkb; ++j) {
