@@ -173,7 +173,11 @@ SVDQ_API svdq_status svdq_attach_lora(svdq_layer_t layer, const void* A, const v
  *   scales  INT4: float [K/64][M_pad] (group scale amax/7, transposed).
  *           NVFP4: uint8 E4M3 in 512-byte atoms, atom (m/128)*(K/64) + k/64,
  *                  byte (m%32)*16 + ((m/32)%4)*4 + (k/16)%4.
- *   T       bf16 [M_pad, rank_pad] = t_scale * (x_hat L1) (columns >= rank are 0)
+ *   T       float [M_pad, rank_pad] = t_scale * (x_hat L1) (columns >= rank are 0):
+ *           the float sum of the bf16 partial products over the shares of K
+ *           that the forward's activation kernel writes to its workspace and
+ *           the GEMM contracts with L2 (this call allocates their buffer on
+ *           `stream` and frees it before returning)
  * with M_pad = M rounded up to a multiple of 128 (rows >= M are zero codes). */
 SVDQ_API svdq_status svdq_quantize_activations(svdq_layer_t layer, const void* X, int M, void* codes, void* scales, void* T,
                                       void* stream);

@@ -9,21 +9,26 @@
 // This kernel reads every X element from HBM once and produces all three in
 // the same pass.
 //
-// Work split: a thread-block cluster of S CTAs owns 64 rows; CTA r of the
-// cluster walks its 1/S share of K in 64-column chunks (S is chosen so the
-// grid covers the SMs once and every cluster is resident). Per chunk:
-//   * warp 17 (one thread) streams the X tile [64 x 64], the L1^T slice
+// Work split: CTA (b, s) owns rows [128 b, 128 b + 128) and the s-th of S
+// equal shares of K, walked in 64-column chunks. S is chosen so that the grid
+// fills the GPU in one wave; the CTAs never wait on one another. Per chunk:
+//   * warp 17 (one thread) streams the X tile [128 x 64], the L1^T slice
 //     [RP x 64] and the inv_s slice into a shared-memory ring with TMA / bulk
-//     copies (128-byte swizzle);
-//   * warps 0-15 (4 rows each) smooth, quantize, store codes and scales, and
-//     write x_hat as a bf16 high part and a bf16 remainder straight into a
-//     tcgen05 K-major operand buffer (128 rows: the MMA's M; rows 64-127 stay
-//     zero and their results are ignored);
+//     copies (128-byte swizzle). The ring is as deep as shared memory allows
+//     (7 stages at RP = 32): X comes from HBM, and the loads in flight are
+//     what sets its bandwidth;
+//   * warps 0-15: each thread owns 16 consecutive elements of one row (a
+//     whole NVFP4 group; a quarter of an INT4 group, whose amax takes two
+//     shuffles). It smooths, quantizes, stores codes and scales, and writes
+//     x_hat as a bf16 high part and a bf16 remainder straight into a tcgen05
+//     K-major operand buffer;
 //   * one thread of warp 16 then issues tcgen05 kind::f16 MMAs
 //     (M = 128, N = RP, bf16 x bf16 -> fp32) of hi and lo against L1 into a
-//     TMEM accumulator, so T's only sizable error is its final bf16 store.
-// At the end the S partial T tiles are reduced through distributed shared
-// memory in a fixed rank order (deterministic), scaled and stored as bf16.
+//     TMEM accumulator, so x_hat enters the product with float accuracy.
+// At the end each CTA stores its partial product over its share of K,
+// scaled by t_scale, as bf16 columns [s RP, (s+1) RP) of T [M_pad, S RP].
+// The GEMM's branch contracts all S partials against L2 in one accumulation,
+// so their sum never makes a pass of its own.
 //
 // Numerics of the quantizer match the CPU oracle operation by operation:
 // every product and quotient is a single IEEE round-to-nearest operation
@@ -38,34 +43,32 @@ namespace svdq {
 
 namespace {
 
-constexpr int kRows = 64;      // rows per cluster
-constexpr int kMmaM = 128;     // tcgen05 M; operand rows >= kRows are zero
-constexpr int kQWarps = 16;    // quantizing warps, 4 rows each
-constexpr int kMmaWarp = kQWarps;      // TMEM owner + MMA issuer
-constexpr int kProdWarp = kQWarps + 1; // TMA producer
+constexpr int kRows = 128;         // rows per CTA (the MMA's M)
+constexpr int kQWarps = 16;        // quantizing warps, 8 rows each
+constexpr int kMmaWarp = kQWarps;  // TMEM owner + MMA issuer
+constexpr int kProdWarp = kQWarps + 1;
 constexpr int kThreads = (kQWarps + 2) * 32;
-constexpr int kPair = 1;               // chunks each quantizing warp processes per iteration
-constexpr int kChunk = 64;     // columns per chunk (one 128-byte swizzle atom of bf16)
-constexpr int kRedCols = 64;   // columns per cluster-reduction pass
+constexpr int kChunk = 64;         // columns per chunk (one 128-byte swizzle atom of bf16)
+constexpr int kMaxSplit = 16;      // K shares per row block (bounds the T partials the GEMM sums)
 
 template <int RP>
 struct K1Shape {
-  static constexpr int kStages = RP <= 64 ? 4 : (RP <= 224 ? 3 : 2);
-  // x_hat operand buffers: phase A runs up to this many chunks ahead of the MMA
-  static constexpr int kABufs = RP <= 128 ? 4 : 3;
+  static constexpr int kABufs = 2;                   // x_hat operand buffers
   static constexpr int kX = kRows * 128;             // X tile of a chunk (bf16, 64 cols)
   static constexpr int kL = RP * 128;                // L1^T slice of a chunk
-  static constexpr int kS = 1024;                    // inv_s slice of a chunk (256 B used, 1 KB keeps alignment)
-  static constexpr int kStage = kX + kL + kS;
-  static constexpr int kAHalf = kMmaM * 128;         // one operand (hi or lo) of a chunk
+  static constexpr int kS = 256;                     // inv_s slice of a chunk
+  static constexpr int kStage = ((kX + kL + kS + 1023) / 1024) * 1024;  // 128-byte-swizzled TMA tiles start 1 KB-aligned
+  static constexpr int kAHalf = kRows * 128;         // one operand (hi or lo) of a chunk
   static constexpr int kA = 2 * kAHalf;              // hi + lo MMA operand of a chunk
+  static constexpr int kBudget = 232448 - 1024 - 512;  // dynamic shared memory, less alignment slack and barriers
+  static constexpr int kStagesFit = (kBudget - kABufs * kA) / kStage;
+  static constexpr int kStages = kStagesFit < 8 ? kStagesFit : 8;
   static constexpr int kAOff = kStages * kStage;
-  static constexpr int kRedOff = kAOff + kABufs * kA;
-  static constexpr int kRedW = RP < kRedCols ? RP : kRedCols;
-  static constexpr int kRed = kRows * kRedW * 4;
-  static constexpr int kBarOff = kRedOff + kRed;
+  static constexpr int kBarOff = kAOff + kABufs * kA;
   static constexpr int kTotal = kBarOff + 256 + 1024;
-  static_assert(kTotal <= 232448, "shared memory budget");
+  static_assert(kStages >= 2 && kTotal <= 232448, "shared memory budget");
+  static_assert(kX % 1024 == 0 && kL % 1024 == 0, "TMA destinations stay 1024-byte aligned");
+  static constexpr int kMinBlocks = 1;
   static constexpr uint32_t kTmemCols = RP <= 32 ? 32 : (RP <= 64 ? 64 : (RP <= 128 ? 128 : 256));
 };
 
@@ -75,123 +78,66 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t cluster_size() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ uint32_t map_peer(uint32_t saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ float4 ld_peer_v4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
-  return v;
-}
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// Quantize NP independent sets of 8 consecutive smoothed values (each one
-// lane's share of a group in a different row or chunk), stage by stage so the
-// NP dependency chains interleave; then store the codes and, from one lane per
-// group, the group scales.
-template <int FMT, int NP>
-__device__ __forceinline__ void quantize_passes(const float (&v)[NP][8], const ActQuantParams& p, const int (&row)[NP],
-                                                const int (&k)[NP], int cs) {
-  float amax[NP];
+// Quantize this thread's 16 consecutive smoothed values v (row `row`, columns
+// k0 .. k0+15) and store their codes and group scale.
+template <int FMT>
+__device__ __forceinline__ void quantize16(const float (&v)[16], const ActQuantParams& p, int row, int k0, int seg) {
+  float m[8];
 #pragma unroll
-  for (int u = 0; u < NP; ++u) {
-    const float m01 = fmaxf(fabsf(v[u][0]), fabsf(v[u][1])), m23 = fmaxf(fabsf(v[u][2]), fabsf(v[u][3]));
-    const float m45 = fmaxf(fabsf(v[u][4]), fabsf(v[u][5])), m67 = fmaxf(fabsf(v[u][6]), fabsf(v[u][7]));
-    amax[u] = fmaxf(fmaxf(m01, m23), fmaxf(m45, m67));
-  }
+  for (int i = 0; i < 8; ++i) m[i] = fmaxf(fabsf(v[2 * i]), fabsf(v[2 * i + 1]));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m[i] = fmaxf(m[i], m[i + 4]);
+  float amax = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
   if (FMT == SVDQ_INT4_G64) {
-    // group of 64 = the 8 lanes sharing (lane >> 3)
+    // a group of 64 = the 4 lanes of this row (lane >> 2 shared)
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    const float safe = amax > 0.f ? amax : 1.f;
+    const float scale = amax > 0.f ? __fdiv_rn(safe, 7.0f) : 0.f;
+    const float inv = __fdiv_rn(7.0f, safe);
+    // |v| <= amax and inv <= (7 / amax)(1 + 2^-24), so |v * inv| rounds to at
+    // most 7: rint already lands in [-7, 7] and the [-8, 7] clamp never acts.
+    // An all-zero group gives v = 0 and codes 0 with the placeholder inv.
+    // The rounding must see the float32-rounded product, so it is rintf on
+    // the product (an add-based round-to-integer would be fused with the
+    // multiply into one FMA and round the exact product instead).
+    uint32_t c[4];
 #pragma unroll
-    for (int o = 1; o <= 4; o <<= 1)
-#pragma unroll
-      for (int u = 0; u < NP; ++u) amax[u] = fmaxf(amax[u], __shfl_xor_sync(0xffffffffu, amax[u], o));
-    float scale[NP], inv[NP];
-#pragma unroll
-    for (int u = 0; u < NP; ++u) {
-      const float safe = amax[u] > 0.f ? amax[u] : 1.f;
-      scale[u] = amax[u] > 0.f ? __fdiv_rn(safe, 7.0f) : 0.f;
-      inv[u] = __fdiv_rn(7.0f, safe);
+    for (int i = 0; i < 4; ++i) {
+      const float2 p01 = __fmul2_rn(make_float2(v[4 * i], v[4 * i + 1]), make_float2(inv, inv));
+      const float2 p23 = __fmul2_rn(make_float2(v[4 * i + 2], v[4 * i + 3]), make_float2(inv, inv));
+      c[i] = cvt_e4m3x2(rintf(p01.x), rintf(p01.y)) | (cvt_e4m3x2(rintf(p23.x), rintf(p23.y)) << 16);
     }
-    uint32_t lo[NP], hi[NP];
-#pragma unroll
-    for (int u = 0; u < NP; ++u) {
-      // |v| <= amax and inv <= (7 / amax)(1 + 2^-24), so |v * inv| rounds to at
-      // most 7: rint already lands in [-7, 7] and the [-8, 7] clamp never acts.
-      // An all-zero group gives v = 0 and codes 0 with the placeholder inv.
-      // The rounding must see the float-rounded product: an add-based
-      // round-to-integer (adding and subtracting 1.5 * 2^23) gets fused with
-      // the multiply into one FMA by the code generator, which rounds the exact
-      // product instead and flips products that land exactly on a half.
-      float q[8];
-#pragma unroll
-      for (int j = 0; j < 8; j += 2) {
-        const float2 pr = __fmul2_rn(make_float2(v[u][j], v[u][j + 1]), make_float2(inv[u], inv[u]));
-        q[j] = rintf(pr.x);
-        q[j + 1] = rintf(pr.y);
-      }
-      lo[u] = cvt_e4m3x2(q[0], q[1]) | (cvt_e4m3x2(q[2], q[3]) << 16);
-      hi[u] = cvt_e4m3x2(q[4], q[5]) | (cvt_e4m3x2(q[6], q[7]) << 16);
-    }
-#pragma unroll
-    for (int u = 0; u < NP; ++u) {
-      *reinterpret_cast<uint2*>(p.codes + static_cast<size_t>(row[u]) * p.K + k[u]) = make_uint2(lo[u], hi[u]);
-      if (cs == 0) reinterpret_cast<float*>(p.scales)[static_cast<size_t>(k[u] >> 6) * p.M_pad + row[u]] = scale[u];
-    }
+    *reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(row) * p.K + k0) = make_uint4(c[0], c[1], c[2], c[3]);
+    if (seg == 0) reinterpret_cast<float*>(p.scales)[static_cast<size_t>(k0 >> 6) * p.M_pad + row] = scale;
   } else {
-    // group of 16 = this lane and its neighbour (lane ^ 1)
+    // a group of 16 = this thread's values
+    const uint32_t sb = cvt_e4m3x2(__fdiv_rn(amax, p.denom), 0.f) & 0xFFu;
+    const float eff = __fmul_rn(e4m3_to_float(sb), p.g_x);
+    const float inv = __frcp_rn(eff != 0.f ? eff : 1.f);
+    float q[2][8];
 #pragma unroll
-    for (int u = 0; u < NP; ++u) amax[u] = fmaxf(amax[u], __shfl_xor_sync(0xffffffffu, amax[u], 1));
-    uint32_t sb[NP];
-    float eff[NP];
-#pragma unroll
-    for (int u = 0; u < NP; ++u) {
-      sb[u] = cvt_e4m3x2(__fdiv_rn(amax[u], p.denom), 0.f) & 0xFFu;
-      eff[u] = __fmul_rn(e4m3_to_float(sb[u]), p.g_x);
-    }
-    uint32_t codes[NP];
-#pragma unroll
-    for (int u = 0; u < NP; ++u) {
-      const float inv = __frcp_rn(eff[u] != 0.f ? eff[u] : 1.f);
-      float q[8];
+    for (int h = 0; h < 2; ++h)
 #pragma unroll
       for (int j = 0; j < 8; j += 2) {
-        const float2 pr = __fmul2_rn(make_float2(v[u][j], v[u][j + 1]), make_float2(inv, inv));
-        q[j] = pr.x;
-        q[j + 1] = pr.y;
+        const float2 pr = __fmul2_rn(make_float2(v[8 * h + j], v[8 * h + j + 1]), make_float2(inv, inv));
+        q[h][j] = pr.x;
+        q[h][j + 1] = pr.y;
       }
-      codes[u] = eff[u] != 0.f ? cvt_e2m1x8(q) : 0u;
-    }
-#pragma unroll
-    for (int u = 0; u < NP; ++u) {
-      *reinterpret_cast<uint32_t*>(p.codes + static_cast<size_t>(row[u]) * (p.K >> 1) + (k[u] >> 1)) = codes[u];
-      if ((cs & 1) == 0) {
-        const int sf = k[u] >> 4;  // scale index along the row
-        const size_t atom = static_cast<size_t>(row[u] >> 7) * (p.K >> 6) + (sf >> 2);
-        const int off = (row[u] & 31) * 16 + ((row[u] >> 5) & 3) * 4 + (sf & 3);
-        reinterpret_cast<uint8_t*>(p.scales)[atom * 512 + off] = static_cast<uint8_t>(sb[u]);
-      }
-    }
+    const uint32_t c0 = eff != 0.f ? cvt_e2m1x8(q[0]) : 0u;
+    const uint32_t c1 = eff != 0.f ? cvt_e2m1x8(q[1]) : 0u;
+    *reinterpret_cast<uint2*>(p.codes + static_cast<size_t>(row) * (p.K >> 1) + (k0 >> 1)) = make_uint2(c0, c1);
+    // scale-factor atom: (row / 128) * (K / 64) + k / 64, byte (row % 32) * 16 + ((row / 32) % 4) * 4 + (k / 16) % 4
+    const size_t atom = static_cast<size_t>(row >> 7) * (p.K >> 6) + (k0 >> 6);
+    const int off = (row & 31) * 16 + ((row >> 5) & 3) * 4 + ((k0 >> 4) & 3);
+    reinterpret_cast<uint8_t*>(p.scales)[atom * 512 + off] = static_cast<uint8_t>(sb);
   }
 }
 
 template <int FMT, int RP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, K1Shape<RP>::kMinBlocks)
     act_quant_kernel(const ActQuantParams p, const __grid_constant__ ActQuantMaps maps) {
   using S = K1Shape<RP>;
   static_assert(RP % 32 == 0 && RP <= 256, "rank padding must be a multiple of 32, at most 256");
@@ -199,20 +145,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);  // [kStages] TMA landed
   uint64_t* empty = full + S::kStages;                             // [kStages] MMA done with the stage
-  uint64_t* aready = empty + S::kStages;                           // [S::kABufs] operand written by warps 0-15
-  uint64_t* afree = aready + S::kABufs;                               // [S::kABufs] MMA done reading the operand
+  uint64_t* aready = empty + S::kStages;                           // [kABufs] operand written by warps 0-15
+  uint64_t* afree = aready + S::kABufs;                            // [kABufs] MMA done reading the operand
   uint64_t* mma_done = afree + S::kABufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t csize = cluster_size();
-  const uint32_t crank = cluster_rank();
-  const int m0 = (blockIdx.x / csize) * kRows;
+  const int split = p.split;
+  const int rb = blockIdx.x / split;
+  const int sh = blockIdx.x % split;  // this CTA's share of K
+  const int m0 = rb * kRows;
   const int nchunks = p.K / kChunk;
-  const int c_begin = static_cast<int>(crank * nchunks / csize);
-  const int c_end = static_cast<int>((crank + 1) * nchunks / csize);
+  const int c_begin = sh * nchunks / split;
+  const int c_end = (sh + 1) * nchunks / split;
   const int nlocal = c_end - c_begin;
 
   if (threadIdx.x == 0) {
@@ -231,16 +178,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, S::kTmemCols);
     tmem_relinquish();
-  }
-  {
-    // operand rows kRows..kMmaM-1 are never written per chunk: clear them once
-    uint4* a = reinterpret_cast<uint4*>(smem + S::kAOff);
-    const int per_half = (kMmaM - kRows) * 128 / 16;
-    for (int i = threadIdx.x; i < 2 * S::kABufs * per_half; i += kThreads) {
-      const int half = i / per_half;  // (buffer, hi/lo)
-      a[(half * S::kAHalf + kRows * 128) / 16 + (i % per_half)] = make_uint4(0, 0, 0, 0);
-    }
-    fence_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -273,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_dense(kFmtF32, kFmtBF16, kFmtBF16, kMmaM, RP);
+      const uint32_t idesc = idesc_dense(kFmtF32, kFmtBF16, kFmtBF16, kRows, RP);
       for (int j = 0; j < nlocal; ++j) {
         const int b = j % S::kABufs;
         if (!mbar_wait(&aready[b], (j / S::kABufs) & 1, abort_flag, p.status)) break;
@@ -296,146 +233,81 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------ quantizing warps
-    const int cs = lane & 7;   // 16-byte column segment of the chunk
-    const int rl = lane >> 3;  // row within a 4-row pass
-    const int r0 = warp * (kRows / kQWarps);  // this warp's rows
-    bool ok = true;
-    for (int j0 = 0; j0 < nlocal && ok; j0 += kPair) {
-      const int npair = min(kPair, nlocal - j0);
-      for (int u = 0; u < npair && ok; ++u) {
-        const int j = j0 + u;
-        ok = mbar_wait(&full[j % S::kStages], (j / S::kStages) & 1, abort_flag, p.status);
-        if (ok && j >= S::kABufs)
-          ok = mbar_wait(&afree[j % S::kABufs], ((j / S::kABufs) & 1) ^ 1, abort_flag, p.status);
+    const int seg = lane & 3;                 // 16-column segment of the chunk
+    const int lrow = warp * 8 + (lane >> 2);  // row within the CTA
+    const int row = m0 + lrow;
+    for (int j = 0; j < nlocal; ++j) {
+      const int s = j % S::kStages;
+      const int b = j % S::kABufs;
+      if (!mbar_wait(&full[s], (j / S::kStages) & 1, abort_flag, p.status)) break;
+      if (j >= S::kABufs && !mbar_wait(&afree[b], ((j / S::kABufs) & 1) ^ 1, abort_flag, p.status)) break;
+      const uint8_t* xt = smem + s * S::kStage;
+      const float4* is4 = reinterpret_cast<const float4*>(xt + S::kX + S::kL) + 4 * seg;
+      const uint32_t phys0 = lrow * 128 + (((2 * seg) ^ (lrow & 7)) * 16);
+      const uint32_t phys1 = lrow * 128 + (((2 * seg + 1) ^ (lrow & 7)) * 16);
+      const uint4 x0 = *reinterpret_cast<const uint4*>(xt + phys0);
+      const uint4 x1 = *reinterpret_cast<const uint4*>(xt + phys1);
+      const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+      float v[16];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float4 is = is4[e];
+        // one IEEE round-to-nearest product per element (packed pairs)
+        const float2 a = __fmul2_rn(make_float2(bf16_lo(w[2 * e]), bf16_hi(w[2 * e])), make_float2(is.x, is.y));
+        const float2 c = __fmul2_rn(make_float2(bf16_lo(w[2 * e + 1]), bf16_hi(w[2 * e + 1])), make_float2(is.z, is.w));
+        v[4 * e] = a.x;
+        v[4 * e + 1] = a.y;
+        v[4 * e + 2] = c.x;
+        v[4 * e + 3] = c.y;
       }
-      if (!ok) break;
-      // The passes of the pair (and of the rows of this warp) are independent:
-      // every stage below runs over all of them, so their chains interleave.
-      constexpr int kPasses = kRows / kQWarps / 4;  // 4-row passes per chunk
-      constexpr int NP = kPair * kPasses;
-      float v[NP][8];
-      int rows[NP], ks[NP];
-      uint8_t* adst[NP];
-      int phys[NP];
+      quantize16<FMT>(v, p, row, (c_begin + j) * kChunk + 16 * seg, seg);
+      // x_hat = hi + lo with hi = bf16(x_hat) and lo = bf16(x_hat - hi) (the
+      // difference is exact in float), in the same 128-byte swizzle as the
+      // TMA tiles: the canonical tcgen05 K-major layout
+      uint32_t h[8], l[8];
 #pragma unroll
-      for (int u = 0; u < kPair; ++u) {
-        const int j = j0 + (u < npair ? u : 0);  // a missing second chunk repeats the first (results unused)
-        const uint8_t* xt = smem + (j % S::kStages) * S::kStage;
-        const float* inv_s = reinterpret_cast<const float*>(xt + S::kX + S::kL) + cs * 8;
-        const float4 is0 = *reinterpret_cast<const float4*>(inv_s);
-        const float4 is1 = *reinterpret_cast<const float4*>(inv_s + 4);
-#pragma unroll
-        for (int i = 0; i < kPasses; ++i) {
-          const int n = u * kPasses + i;
-          const int lrow = r0 + 4 * i + rl;
-          phys[n] = lrow * 128 + (cs ^ (lrow & 7)) * 16;
-          rows[n] = m0 + lrow;
-          ks[n] = (c_begin + j) * kChunk + cs * 8;
-          adst[n] = smem + S::kAOff + (j % S::kABufs) * S::kA;
-          const uint4 xv = *reinterpret_cast<const uint4*>(xt + phys[n]);
-          const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
-          const float is[8] = {is0.x, is0.y, is0.z, is0.w, is1.x, is1.y, is1.z, is1.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            // one IEEE round-to-nearest product per element (packed pair)
-            const float2 pr = __fmul2_rn(make_float2(bf16_lo(w[e]), bf16_hi(w[e])), make_float2(is[2 * e], is[2 * e + 1]));
-            v[n][2 * e] = pr.x;
-            v[n][2 * e + 1] = pr.y;
-          }
-        }
+      for (int e = 0; e < 8; ++e) {
+        h[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+        const float2 d = __fadd2_rn(make_float2(v[2 * e], v[2 * e + 1]), make_float2(-bf16_lo(h[e]), -bf16_hi(h[e])));
+        l[e] = pack_bf16x2(d.x, d.y);
       }
-      if (npair == kPair) {
-        quantize_passes<FMT, NP>(v, p, rows, ks, cs);
-      } else {
-        float v1[kPasses][8];
-        int rows1[kPasses], ks1[kPasses];
-#pragma unroll
-        for (int n = 0; n < kPasses; ++n) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) v1[n][e] = v[n][e];
-          rows1[n] = rows[n];
-          ks1[n] = ks[n];
-        }
-        quantize_passes<FMT, kPasses>(v1, p, rows1, ks1, cs);
-      }
-#pragma unroll
-      for (int n = 0; n < NP; ++n) {
-        if (n < npair * kPasses) {
-          uint32_t h[4], l[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            h[e] = pack_bf16x2(v[n][2 * e], v[n][2 * e + 1]);  // high parts, one packed conversion
-            // the remainders are exact in float: v - bf16(v) has at most 16 significant bits
-            const float2 d = __fadd2_rn(make_float2(v[n][2 * e], v[n][2 * e + 1]),
-                                        make_float2(-bf16_lo(h[e]), -bf16_hi(h[e])));
-            l[e] = pack_bf16x2(d.x, d.y);
-          }
-          // same 128-byte swizzle as the TMA tiles: the canonical tcgen05 K-major layout
-          *reinterpret_cast<uint4*>(adst[n] + phys[n]) = make_uint4(h[0], h[1], h[2], h[3]);
-          *reinterpret_cast<uint4*>(adst[n] + S::kAHalf + phys[n]) = make_uint4(l[0], l[1], l[2], l[3]);
-        }
-      }
+      uint8_t* ad = smem + S::kAOff + b * S::kA;
+      *reinterpret_cast<uint4*>(ad + phys0) = make_uint4(h[0], h[1], h[2], h[3]);
+      *reinterpret_cast<uint4*>(ad + phys1) = make_uint4(h[4], h[5], h[6], h[7]);
+      *reinterpret_cast<uint4*>(ad + S::kAHalf + phys0) = make_uint4(l[0], l[1], l[2], l[3]);
+      *reinterpret_cast<uint4*>(ad + S::kAHalf + phys1) = make_uint4(l[4], l[5], l[6], l[7]);
       fence_async_smem();  // make the generic-proxy writes visible to the tensor core
       __syncwarp();
-      if (lane == 0)
-        for (int u = 0; u < npair; ++u) mbar_arrive(&aready[(j0 + u) % S::kABufs]);
+      if (lane == 0) mbar_arrive(&aready[b]);
     }
   }
 
-  // ------------------------------------------------ cluster reduction of T
+  // ------------------------------------------------ this CTA's share of T
   {
     volatile int no_abort = 0;
     mbar_wait(mma_done, 0, &no_abort, nullptr);
   }
   tc_fence_after();
-  const bool healthy = !*abort_flag;
-  float* red = reinterpret_cast<float*>(smem + S::kRedOff);
-  const uint32_t red_s = smem_u32(red);
-  for (int c0 = 0; c0 < RP; c0 += S::kRedW) {
-    // 1. each CTA parks its partial [128 x kRedW] fp32 in its own shared memory
-    if (warp < 8 && healthy) {
-      const int q = warp & 3;
-      const int half = warp >> 2;
-      if (half * 32 < S::kRedW && q * 32 < kRows) {
-        uint32_t r[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + c0 + half * 32, r);
-        tmem_ld_wait();
-        float* dst = red + (32 * q + lane) * S::kRedW + half * 32;
+  if (warp < 4 && !*abort_flag) {
+    // warp q may read TMEM lanes 32q .. 32q+31: rows 32q .. 32q+31 of the CTA
+    const int r = m0 + 32 * warp + lane;
+    __nv_bfloat16* dst = p.T + static_cast<size_t>(r) * p.TP + sh * RP;
+#pragma unroll 1
+    for (int c0 = 0; c0 < RP; c0 += 32) {
+      uint32_t acc[32];
+      tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + c0, acc);
+      tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(dst + e) = make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
-                                                            __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
-      }
-    }
-    cluster_sync();
-    // 2. CTA r sums rows [r*128/S, (r+1)*128/S) over the cluster, rank 0 first
-    if (healthy) {
-      const int rows_per = kRows / static_cast<int>(csize);
-      const int rbeg = static_cast<int>(crank) * rows_per;
-      const int nvec = rows_per * (S::kRedW / 4);
-      for (int i = threadIdx.x; i < nvec; i += kThreads) {
-        const int row = rbeg + i / (S::kRedW / 4);
-        const int col = (i % (S::kRedW / 4)) * 4;
-        const uint32_t off = static_cast<uint32_t>((row * S::kRedW + col) * 4);
-        float4 part[8];
-#pragma unroll
-        for (uint32_t pr = 0; pr < 8; ++pr)
-          if (pr < csize) part[pr] = ld_peer_v4(map_peer(red_s + off, pr));
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (uint32_t pr = 0; pr < 8; ++pr)
-          if (pr < csize) {  // fixed rank order: deterministic sums
-            acc.x += part[pr].x;
-            acc.y += part[pr].y;
-            acc.z += part[pr].z;
-            acc.w += part[pr].w;
-          }
+      for (int e = 0; e < 32; e += 8) {
         const float sc = p.t_scale;
-        uint2 out = make_uint2(pack_bf16x2(acc.x * sc, acc.y * sc), pack_bf16x2(acc.z * sc, acc.w * sc));
-        *reinterpret_cast<uint2*>(p.T + static_cast<size_t>(m0 + row) * RP + c0 + col) = out;
+        const uint4 o = make_uint4(
+            pack_bf16x2(__uint_as_float(acc[e]) * sc, __uint_as_float(acc[e + 1]) * sc),
+            pack_bf16x2(__uint_as_float(acc[e + 2]) * sc, __uint_as_float(acc[e + 3]) * sc),
+            pack_bf16x2(__uint_as_float(acc[e + 4]) * sc, __uint_as_float(acc[e + 5]) * sc),
+            pack_bf16x2(__uint_as_float(acc[e + 6]) * sc, __uint_as_float(acc[e + 7]) * sc));
+        *reinterpret_cast<uint4*>(dst + c0 + e) = o;
       }
     }
-    cluster_sync();  // peers are done reading before the buffer is reused or the CTA exits
   }
 
   // ------------------------------------------------ teardown
@@ -447,32 +319,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Cluster size: the largest power of two <= 8 whose clusters all fit on the
-// GPU at once (cluster placement, not just the SM count, decides that) and
-// that leaves every CTA at least one chunk.
-template <class Kern>
-int choose_split(Kern kern, int smem, int row_blocks, int nchunks) {
-  int best = 1;
-  for (int s = 2; s <= 8 && s <= nchunks; s *= 2) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(row_blocks * s, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = s;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) {
-      cudaGetLastError();
-      break;
-    }
-    if (clusters >= row_blocks) best = s;
+// Sum of the S bf16 partials of T into float [M_pad, RP] (introspection only).
+__global__ void t_partials_sum_kernel(const __nv_bfloat16* Tp, int M_pad, int RP, int split, float* out) {
+  const size_t n = static_cast<size_t>(M_pad) * RP;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t r = i / RP, c = i % RP;
+    float acc = 0.f;
+    for (int s = 0; s < split; ++s) acc += __bfloat162float(Tp[r * static_cast<size_t>(split) * RP + s * RP + c]);
+    out[i] = acc;
   }
-  return best;
 }
 
 template <int FMT, int RP>
@@ -483,31 +339,38 @@ cudaError_t launch_rp(const ActQuantParams& p, const ActQuantMaps& maps, cudaStr
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
-    if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const int row_blocks = p.M_pad / kRows;
-  static int cached_rb = -1, cached_k = -1, cached_split = 1;
-  if (row_blocks != cached_rb || p.K != cached_k) {
-    cached_split = choose_split(kern, S::kTotal, row_blocks, p.K / kChunk);
-    cached_rb = row_blocks;
-    cached_k = p.K;
+  act_quant_kernel<FMT, RP><<<(p.M_pad / kRows) * p.split, kThreads, S::kTotal, stream>>>(p, maps);
+  return cudaGetLastError();
+}
+
+template <int FMT, int RP>
+int resident_ctas() {
+  using S = K1Shape<RP>;
+  auto kern = act_quant_kernel<FMT, RP>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal) != cudaSuccess) return 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, S::kTotal) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    return 1;
   }
-  const int split = cached_split;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(row_blocks * split, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = S::kTotal;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = split;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, p, maps);
+  return n;
+}
+
+template <int FMT>
+int resident_fmt(int rp) {
+  switch (rp) {
+    case 32: return resident_ctas<FMT, 32>();
+    case 64: return resident_ctas<FMT, 64>();
+    case 96: return resident_ctas<FMT, 96>();
+    case 128: return resident_ctas<FMT, 128>();
+    case 160: return resident_ctas<FMT, 160>();
+    case 192: return resident_ctas<FMT, 192>();
+    case 224: return resident_ctas<FMT, 224>();
+    case 256: return resident_ctas<FMT, 256>();
+    default: return 1;
+  }
 }
 
 template <int FMT>
@@ -529,11 +392,35 @@ cudaError_t launch_fmt(const ActQuantParams& p, const ActQuantMaps& maps, int rp
 
 int act_quant_box_rows() { return kRows; }
 
+int act_quant_split(int M_pad, int K, int fmt, int rp, int sms) {
+  // CTAs that fit on the GPU at once, divided among the 64-row blocks; each
+  // CTA keeps at least one chunk, and at most kMaxSplit partials are summed.
+  // resident CTAs per SM for (format, rank padding), queried once per process
+  static int cache[2][9] = {};
+  const int fi = fmt == SVDQ_INT4_G64 ? 0 : 1, ri = rp / 32;
+  if (ri < 1 || ri > 8) return 1;
+  if (cache[fi][ri] == 0)
+    cache[fi][ri] = fmt == SVDQ_INT4_G64 ? resident_fmt<SVDQ_INT4_G64>(rp) : resident_fmt<SVDQ_NVFP4_G16>(rp);
+  const int per_sm = cache[fi][ri];
+  const int row_blocks = M_pad / kRows;
+  int split = (sms * per_sm) / row_blocks;
+  const int nchunks = K / kChunk;
+  if (split > nchunks) split = nchunks;
+  if (split > kMaxSplit) split = kMaxSplit;
+  return split < 1 ? 1 : split;
+}
+
 cudaError_t launch_act_quant(const ActQuantParams& p, const ActQuantMaps& maps, int fmt, int rp,
                              cudaStream_t stream) {
-  if (p.M_pad % 128 != 0 || p.K % 128 != 0) return cudaErrorInvalidValue;
+  if (p.M_pad % 128 != 0 || p.K % 128 != 0 || p.split < 1 || p.TP != p.split * rp) return cudaErrorInvalidValue;
   if (fmt == SVDQ_INT4_G64) return launch_fmt<SVDQ_INT4_G64>(p, maps, rp, stream);
   return launch_fmt<SVDQ_NVFP4_G16>(p, maps, rp, stream);
+}
+
+cudaError_t launch_t_partials_sum(const __nv_bfloat16* Tp, int M_pad, int RP, int split, float* out,
+                                  cudaStream_t stream) {
+  t_partials_sum_kernel<<<148, 256, 0, stream>>>(Tp, M_pad, RP, split, out);
+  return cudaGetLastError();
 }
 
 }  // namespace svdq

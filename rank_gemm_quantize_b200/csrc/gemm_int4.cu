@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_tiles = (p.M_pad / kBM) * n_blocks;
   const int n_groups = p.K / 64;
   const int n_main = p.K / kBK;
-  const int n_lr = p.RP / 32;
+  const int n_lr = p.TP / 32;  // branch k-tiles: every split partial of T
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int c = k - n_main;  // 32-column slice of the branch
             mbar_arrive_expect_tx(&full[s], kBM * 64 + kBN * 64);
             tma_load_2d(st, &maps.t, &full[s], c * 32, m0);
-            tma_load_2d(st + L::kA, &maps.l2, &full[s], c * 32, n0);
+            tma_load_2d(st + L::kA, &maps.l2, &full[s], (c % (p.RP / 32)) * 32, n0);
           }
         }
       }

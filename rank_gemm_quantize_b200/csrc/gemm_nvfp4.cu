@@ -16,8 +16,9 @@
 // Warp roles (10 warps):
 //   warp 0  producer: for each tile, a bulk copy of the bias slice, then the
 //           k-tiles (A and B codes by TMA, their scale-factor atoms by bulk
-//           copy; four copies in flight per stage) followed by RP/32 branch
-//           k-tiles (a 32-column slice of T' and of L2^T), through a 4-stage
+//           copy; four copies in flight per stage) followed by the branch
+//           k-tiles (a 32-column slice of one of the activation kernel's
+//           partials of T' and the matching slice of L2^T), through a 4-stage
 //           shared-memory ring;
 //   warp 1  TMEM owner and MMA issuer (one thread): scale factors to TMEM
 //           with tcgen05.cp, then 4 block-scaled MMAs per k-tile, 2 kind::f16
@@ -86,7 +87,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_tiles = (p.M_pad / kBM) * n_blocks;
   const int kb_total = p.K / 64;
   const int n_main = (p.K + 255) / 256;
-  const int n_lr = p.RP / 32;
+  const int n_lr = p.TP / 32;  // branch k-tiles: every split partial of T
   const int n_items = n_main + n_lr;
 
   if (threadIdx.x == 0) {
@@ -156,7 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int c = k - n_main;  // 32-column slice of the branch
             mbar_arrive_expect_tx(&full[s], kBM * 64 + kBN * 64);
             tma_load_2d(st, &maps.t, &full[s], c * 32, m0);
-            tma_load_2d(st + L::kA, &maps.l2, &full[s], c * 32, n0);
+            tma_load_2d(st + L::kA, &maps.l2, &full[s], (c % (p.RP / 32)) * 32, n0);
           }
         }
       }

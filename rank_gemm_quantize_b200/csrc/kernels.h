@@ -17,7 +17,8 @@ struct ActQuantParams {
   const __nv_bfloat16* L1T;  // [RP, K]: transposed, zero-padded down-projection factor
   uint8_t* codes;          // INT4: [M_pad, K] E4M3 bytes of the integer codes; NVFP4: [M_pad, K/2] packed E2M1
   void* scales;            // INT4: float [K/64][M_pad]; NVFP4: scale-factor atoms [M_pad/128][K/64][512]
-  __nv_bfloat16* T;        // [M_pad, RP] bf16, multiplied by t_scale
+  __nv_bfloat16* T;        // [M_pad, TP] bf16: split partials of t_scale * (x_hat L1), RP columns each
+  int split, TP;           // K shares per 64-row block (from act_quant_split) and TP = split * RP
   float g_x;               // NVFP4 activation tensor scale
   float denom;             // NVFP4: fp32(6 * g_x)
   float t_scale;           // 1 (INT4) or 1 / (g_x g_w) (NVFP4)
@@ -28,11 +29,17 @@ struct ActQuantMaps {
   CUtensorMap l1t;  // L1T [RP, K] bf16, box {64, RP}, 128-byte swizzle
 };
 int act_quant_box_rows();
+// K shares per 64-row block for M_pad rows: the grid fills the GPU in one wave.
+int act_quant_split(int M_pad, int K, int fmt, int rp, int sms);
 cudaError_t launch_act_quant(const ActQuantParams& p, const ActQuantMaps& maps, int fmt, int rp, cudaStream_t stream);
+// out[m, c] = sum over the split partials of T (float), for introspection.
+cudaError_t launch_t_partials_sum(const __nv_bfloat16* Tp, int M_pad, int RP, int split, float* out,
+                                  cudaStream_t stream);
 
 // ---------------------------------------------------------------- GEMMs
 struct GemmParams {
   int M, N, K, RP;
+  int TP;                      // columns of T: the activation kernel's split partials, RP each
   __nv_bfloat16* Y;            // [M, N]
   const __nv_bfloat16* bias;   // [N_pad], zero beyond N
   const void* sa;              // activation scales (layout of ActQuantParams::scales)
@@ -44,7 +51,7 @@ struct GemmParams {
 struct GemmMaps {
   CUtensorMap a;   // activation codes
   CUtensorMap b;   // weight codes
-  CUtensorMap t;   // T [M_pad, RP] bf16
+  CUtensorMap t;   // T [M_pad, TP] bf16 (partials; each is contracted with L2)
   CUtensorMap l2;  // L2T [N_pad, RP] bf16
 };
 int gemm_nvfp4_bn();  // tile width (rows of the weight box) of each GEMM

@@ -29,7 +29,8 @@ void set_last_error(const std::string& msg);
 namespace {
 
 // Largest workspace the array holds: enough for M x K = 4608 x 3072 in either
-// format at rank <= 32 (about 15.3 MiB for INT4, 8.2 MiB for NVFP4).
+// format at rank <= 32 (about 15.5 MiB for INT4, 8.4 MiB for NVFP4, with the
+// activation kernel's partials of T).
 constexpr size_t kScratchBytes = size_t(16) << 20;
 
 constexpr int kMaxDevices = 64;

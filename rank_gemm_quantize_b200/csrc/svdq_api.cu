@@ -106,6 +106,7 @@ struct MapCache {
 
 struct WsLayout {
   int M_pad;
+  int split, TP;  // activation-kernel K shares and the width of T (split * RP)
   size_t codes, scales, T, total;
 };
 
@@ -113,6 +114,7 @@ struct WsLayout {
 
 struct svdq_layer {
   int device = 0;
+  int sms = 148;  // SM count of the device, read at preparation
   svdq_config cfg{};
   int K = 0, N = 0, N_pad = 0, rank = 0, RP = 0;
   int fmt = 0;
@@ -141,8 +143,10 @@ WsLayout ws_layout(const svdq_layer* h, int M) {
                                                 : static_cast<size_t>(w.M_pad / 128) * (h->K / 64) * 512;
   w.codes = 0;
   w.scales = align256(cbytes);
+  w.split = act_quant_split(w.M_pad, h->K, h->fmt, h->RP, h->sms);
+  w.TP = w.split * h->RP;
   w.T = w.scales + align256(sbytes);
-  w.total = w.T + align256(static_cast<size_t>(w.M_pad) * h->RP * 2);
+  w.total = w.T + align256(static_cast<size_t>(w.M_pad) * w.TP * 2);
   return w;
 }
 
@@ -310,6 +314,10 @@ svdq_status start_prepare(const svdq_config* cfg, const void* W, const void* bia
     return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
   svdq_layer* h = new svdq_layer();
   cudaGetDevice(&h->device);
+  if (cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess || h->sms < 1) {
+    cudaGetLastError();
+    h->sms = 148;
+  }
   h->cfg = *cfg;
   h->K = cfg->K;
   h->N = cfg->N;
@@ -423,8 +431,10 @@ svdq_status svd_factors(svdq_layer* h, const float* W_hat, __nv_bfloat16* L1, __
 }
 
 svdq_status launch_k1(svdq_layer* h, const void* X, int M, uint8_t* codes, void* scales, __nv_bfloat16* T,
-                      cudaStream_t st) {
+                      const WsLayout& w, cudaStream_t st) {
   ActQuantParams p{};
+  p.split = w.split;
+  p.TP = w.TP;
   p.X = static_cast<const __nv_bfloat16*>(X);
   p.M = M;
   p.K = h->K;
@@ -546,7 +556,7 @@ svdq_status forward_impl(svdq_layer* h, const void* X, int M, void* Y, void* wor
   void* scales = base + w.scales;
   __nv_bfloat16* T = reinterpret_cast<__nv_bfloat16*>(base + w.T);
   if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[0]), st));
-  svdq_status e = launch_k1(h, X, M, codes, scales, T, st);
+  svdq_status e = launch_k1(h, X, M, codes, scales, T, w, st);
   if (e) return e;
   if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[1]), st));
   auto* we = h->ws_maps.find(workspace, M);
@@ -556,7 +566,7 @@ svdq_status forward_impl(svdq_layer* h, const void* X, int M, void* Y, void* wor
     const uint64_t row = i4 ? h->K : h->K / 2;
     if (!make_map(&we->a, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, row, w.M_pad, row, 128, 128,
                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&we->b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, h->RP, w.M_pad, static_cast<uint64_t>(h->RP) * 2, 32,
+        !make_map(&we->b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, w.TP, w.M_pad, static_cast<uint64_t>(w.TP) * 2, 32,
                   128, CU_TENSOR_MAP_SWIZZLE_64B)) {
       we->key = nullptr;
       return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (activations) failed");
@@ -567,6 +577,7 @@ svdq_status forward_impl(svdq_layer* h, const void* X, int M, void* Y, void* wor
   p.N = h->N;
   p.K = h->K;
   p.RP = h->RP;
+  p.TP = w.TP;
   p.Y = static_cast<__nv_bfloat16*>(Y);
   p.bias = h->bias;
   p.sa = scales;
@@ -607,8 +618,19 @@ svdq_status svdq_quantize_activations(svdq_layer_t h, const void* X, int M, void
   if (!X || !codes || !scales || !T || M < 1) return fail(SVDQ_ERR_INVALID_ARG, "NULL pointer or M < 1");
   if (!aligned16(X) || !aligned16(codes) || !aligned16(scales) || !aligned16(T))
     return fail(SVDQ_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
-  return launch_k1(h, X, M, static_cast<uint8_t*>(codes), scales, static_cast<__nv_bfloat16*>(T),
-                   static_cast<cudaStream_t>(stream));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const WsLayout w = ws_layout(h, M);
+  // the forward keeps T as split partials; this call returns their float sum
+  void* Tp = nullptr;
+  cudaError_t ce = cudaMallocAsync(&Tp, static_cast<size_t>(w.M_pad) * w.TP * 2, st);
+  if (ce != cudaSuccess) return fail(SVDQ_ERR_OOM, std::string("T partials: ") + cudaGetErrorString(ce));
+  svdq_status e = launch_k1(h, X, M, static_cast<uint8_t*>(codes), scales, static_cast<__nv_bfloat16*>(Tp), w, st);
+  if (e == SVDQ_OK) {
+    ce = launch_t_partials_sum(static_cast<const __nv_bfloat16*>(Tp), w.M_pad, h->RP, w.split, static_cast<float*>(T), st);
+    if (ce != cudaSuccess) e = fail(SVDQ_ERR_CUDA, std::string("T partial sum: ") + cudaGetErrorString(ce));
+  }
+  cudaFreeAsync(Tp, st);
+  return e;
 }
 
 svdq_status svdq_attach_lora(svdq_layer_t h, const void* A, const void* B, int r_l, float scale, void* stream) {
