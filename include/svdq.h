@@ -145,11 +145,11 @@ SVDQ_API svdq_status svdq_linear_forward_profiled(svdq_layer_t layer, const void
  * whose device memory belongs to their own allocator and may not be grown
  * behind its back, or latency-critical loops where an allocation may
  * synchronize the device. The pages describe no such call; it exists for
- * these callers only. The workspace is a fixed 16 MiB scratch array inside
+ * these callers only. The workspace is a fixed 32 MiB scratch array inside
  * the library's device image (held by every GPU that loads the library until
  * the process exits); the caller passes only X and Y. Nothing is allocated
  * and nothing needs clearing: the first kernel overwrites every byte the
- * second one reads. Layers whose workspace for M rows exceeds 16 MiB are
+ * second one reads. Layers whose workspace for M rows exceeds 32 MiB are
  * refused with SVDQ_ERR_INVALID_ARG (svdq_workspace_size gives the need).
  * The first call on a device looks up the array's device address (set-up, once
  * per device, with that device current); make that first call before any
@@ -173,11 +173,10 @@ SVDQ_API svdq_status svdq_attach_lora(svdq_layer_t layer, const void* A, const v
  *   scales  INT4: float [K/64][M_pad] (group scale amax/7, transposed).
  *           NVFP4: uint8 E4M3 in 512-byte atoms, atom (m/128)*(K/64) + k/64,
  *                  byte (m%32)*16 + ((m/32)%4)*4 + (k/16)%4.
- *   T       float [M_pad, rank_pad] = t_scale * (x_hat L1) (columns >= rank are 0):
- *           the float sum of the bf16 partial products over the shares of K
- *           that the forward's activation kernel writes to its workspace and
- *           the GEMM contracts with L2 (this call allocates their buffer on
- *           `stream` and frees it before returning)
+ *   T       bf16 [M_pad, rank_pad] = t_scale * (x_hat L1) (columns >= rank are 0)
+ * The activation kernel splits K into shares whose float partial products it
+ * sums in share order; this call allocates their scratch buffer on `stream`
+ * and frees it before returning (the forward keeps it in its workspace).
  * with M_pad = M rounded up to a multiple of 128 (rows >= M are zero codes). */
 SVDQ_API svdq_status svdq_quantize_activations(svdq_layer_t layer, const void* X, int M, void* codes, void* scales, void* T,
                                       void* stream);

@@ -229,7 +229,7 @@ class Layer:
         else:
             codes = torch.empty(M_pad, K // 2, dtype=torch.uint8, device=dev)
             scales = torch.empty(M_pad // 128 * (K // 64) * 512, dtype=torch.uint8, device=dev)
-        T = torch.empty(M_pad, info.rank_pad, dtype=torch.float32, device=dev)
+        T = torch.empty(M_pad, info.rank_pad, dtype=torch.bfloat16, device=dev)
         _check(lib().svdq_quantize_activations(self._h, _ptr(X), M, _ptr(codes), _ptr(scales), _ptr(T),
                                                _stream(stream)))
         return codes, scales, T

@@ -25,10 +25,12 @@
 //   * one thread of warp 16 then issues tcgen05 kind::f16 MMAs
 //     (M = 128, N = RP, bf16 x bf16 -> fp32) of hi and lo against L1 into a
 //     TMEM accumulator, so x_hat enters the product with float accuracy.
-// At the end each CTA stores its partial product over its share of K,
-// scaled by t_scale, as bf16 columns [s RP, (s+1) RP) of T [M_pad, S RP].
-// The GEMM's branch contracts all S partials against L2 in one accumulation,
-// so their sum never makes a pass of its own.
+// At the end each CTA parks its float partial product over its share of K in
+// the workspace and counts itself in on its row block's arrival counter; the
+// last of the S CTAs to arrive sums the S partials in share order (the same
+// sum whatever the arrival order), scales by t_scale, stores T as bf16 and
+// resets the counter for the next launch. With S = 1 the CTA stores T
+// directly.
 //
 // Numerics of the quantizer match the CPU oracle operation by operation:
 // every product and quotient is a single IEEE round-to-nearest operation
@@ -49,7 +51,7 @@ constexpr int kMmaWarp = kQWarps;  // TMEM owner + MMA issuer
 constexpr int kProdWarp = kQWarps + 1;
 constexpr int kThreads = (kQWarps + 2) * 32;
 constexpr int kChunk = 64;         // columns per chunk (one 128-byte swizzle atom of bf16)
-constexpr int kMaxSplit = 16;      // K shares per row block (bounds the T partials the GEMM sums)
+constexpr int kMaxSplit = 16;      // K shares per row block (bounds the partials the last CTA sums)
 
 template <int RP>
 struct K1Shape {
@@ -150,6 +152,7 @@ __global__ void __launch_bounds__(kThreads, K1Shape<RP>::kMinBlocks)
   uint64_t* mma_done = afree + S::kABufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* is_last = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -288,24 +291,91 @@ __global__ void __launch_bounds__(kThreads, K1Shape<RP>::kMinBlocks)
     mbar_wait(mma_done, 0, &no_abort, nullptr);
   }
   tc_fence_after();
-  if (warp < 4 && !*abort_flag) {
-    // warp q may read TMEM lanes 32q .. 32q+31: rows 32q .. 32q+31 of the CTA
-    const int r = m0 + 32 * warp + lane;
-    __nv_bfloat16* dst = p.T + static_cast<size_t>(r) * p.TP + sh * RP;
+  const bool healthy = !*abort_flag;
+  // warp q may read TMEM lanes 32q .. 32q+31: rows 32q .. 32q+31 of the CTA
+  const int r = m0 + 32 * warp + lane;
+  const float sc = p.t_scale;
+  if (split == 1) {
+    if (warp < 4 && healthy) {
 #pragma unroll 1
-    for (int c0 = 0; c0 < RP; c0 += 32) {
-      uint32_t acc[32];
-      tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + c0, acc);
-      tmem_ld_wait();
+      for (int c0 = 0; c0 < RP; c0 += 32) {
+        uint32_t acc[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + c0, acc);
+        tmem_ld_wait();
 #pragma unroll
-      for (int e = 0; e < 32; e += 8) {
-        const float sc = p.t_scale;
-        const uint4 o = make_uint4(
-            pack_bf16x2(__uint_as_float(acc[e]) * sc, __uint_as_float(acc[e + 1]) * sc),
-            pack_bf16x2(__uint_as_float(acc[e + 2]) * sc, __uint_as_float(acc[e + 3]) * sc),
-            pack_bf16x2(__uint_as_float(acc[e + 4]) * sc, __uint_as_float(acc[e + 5]) * sc),
-            pack_bf16x2(__uint_as_float(acc[e + 6]) * sc, __uint_as_float(acc[e + 7]) * sc));
-        *reinterpret_cast<uint4*>(dst + c0 + e) = o;
+        for (int e = 0; e < 32; e += 8) {
+          const uint4 o = make_uint4(
+              pack_bf16x2(__uint_as_float(acc[e]) * sc, __uint_as_float(acc[e + 1]) * sc),
+              pack_bf16x2(__uint_as_float(acc[e + 2]) * sc, __uint_as_float(acc[e + 3]) * sc),
+              pack_bf16x2(__uint_as_float(acc[e + 4]) * sc, __uint_as_float(acc[e + 5]) * sc),
+              pack_bf16x2(__uint_as_float(acc[e + 6]) * sc, __uint_as_float(acc[e + 7]) * sc));
+          *reinterpret_cast<uint4*>(p.T + static_cast<size_t>(r) * RP + c0 + e) = o;
+        }
+      }
+    }
+  } else {
+    if (warp < 4) {
+      // park this share's partial; a CTA that gave up parks zeros, so the
+      // arrival count stays right and the status word reports the failure
+      float* dst = p.Tpart + (static_cast<size_t>(sh) * p.M_pad + r) * RP;
+#pragma unroll 1
+      for (int c0 = 0; c0 < RP; c0 += 32) {
+        uint32_t acc[32];
+        if (healthy) {
+          tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + c0, acc);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) acc[e] = 0u;
+        }
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(dst + c0 + e) = make_float4(__uint_as_float(acc[e]), __uint_as_float(acc[e + 1]),
+                                                                 __uint_as_float(acc[e + 2]), __uint_as_float(acc[e + 3]));
+      }
+      __threadfence();  // the partial is visible device-wide before this CTA counts itself in
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const int prev = atomicAdd(p.counters + rb, 1);
+      const int last = prev == split - 1;
+      if (last) p.counters[rb] = 0;  // every share has arrived: ready for the next launch
+      *is_last = last;
+    }
+    __syncthreads();
+    if (*is_last && warp < kQWarps) {
+      __threadfence();  // acquire side: the other shares' partials are visible
+      // all quantizing threads sum: one 8-column slice of one row per item,
+      // four shares' loads in flight at a time, shares added in order
+      constexpr int kSlices = RP / 8;
+#pragma unroll 1
+      for (int item = threadIdx.x; item < kRows * kSlices; item += kQWarps * 32) {
+        const int rr = m0 + item / kSlices;
+        const int c0 = (item % kSlices) * 8;
+        const float* src = p.Tpart + static_cast<size_t>(rr) * RP + c0;
+        const size_t stride = static_cast<size_t>(p.M_pad) * RP;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+        for (int t0 = 0; t0 < split; t0 += 4) {
+          float4 u[4], w[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            if (t0 + t < split) {
+              u[t] = __ldcg(reinterpret_cast<const float4*>(src + (t0 + t) * stride));
+              w[t] = __ldcg(reinterpret_cast<const float4*>(src + (t0 + t) * stride + 4));
+            }
+          }
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            if (t0 + t < split) {  // share order: the same sum whatever the arrival order
+              acc[0] += u[t].x; acc[1] += u[t].y; acc[2] += u[t].z; acc[3] += u[t].w;
+              acc[4] += w[t].x; acc[5] += w[t].y; acc[6] += w[t].z; acc[7] += w[t].w;
+            }
+          }
+        }
+        const uint4 o = make_uint4(pack_bf16x2(acc[0] * sc, acc[1] * sc), pack_bf16x2(acc[2] * sc, acc[3] * sc),
+                                   pack_bf16x2(acc[4] * sc, acc[5] * sc), pack_bf16x2(acc[6] * sc, acc[7] * sc));
+        *reinterpret_cast<uint4*>(p.T + static_cast<size_t>(rr) * RP + c0) = o;
       }
     }
   }
@@ -316,18 +386,6 @@ __global__ void __launch_bounds__(kThreads, K1Shape<RP>::kMinBlocks)
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, S::kTmemCols);
-  }
-}
-
-// Sum of the S bf16 partials of T into float [M_pad, RP] (introspection only).
-__global__ void t_partials_sum_kernel(const __nv_bfloat16* Tp, int M_pad, int RP, int split, float* out) {
-  const size_t n = static_cast<size_t>(M_pad) * RP;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const size_t r = i / RP, c = i % RP;
-    float acc = 0.f;
-    for (int s = 0; s < split; ++s) acc += __bfloat162float(Tp[r * static_cast<size_t>(split) * RP + s * RP + c]);
-    out[i] = acc;
   }
 }
 
@@ -412,15 +470,11 @@ int act_quant_split(int M_pad, int K, int fmt, int rp, int sms) {
 
 cudaError_t launch_act_quant(const ActQuantParams& p, const ActQuantMaps& maps, int fmt, int rp,
                              cudaStream_t stream) {
-  if (p.M_pad % 128 != 0 || p.K % 128 != 0 || p.split < 1 || p.TP != p.split * rp) return cudaErrorInvalidValue;
+  if (p.M_pad % 128 != 0 || p.K % 128 != 0 || p.split < 1 || p.M_pad / kRows > kMaxRowBlocks ||
+      (p.split > 1 && (!p.Tpart || !p.counters)))
+    return cudaErrorInvalidValue;
   if (fmt == SVDQ_INT4_G64) return launch_fmt<SVDQ_INT4_G64>(p, maps, rp, stream);
   return launch_fmt<SVDQ_NVFP4_G16>(p, maps, rp, stream);
-}
-
-cudaError_t launch_t_partials_sum(const __nv_bfloat16* Tp, int M_pad, int RP, int split, float* out,
-                                  cudaStream_t stream) {
-  t_partials_sum_kernel<<<148, 256, 0, stream>>>(Tp, M_pad, RP, split, out);
-  return cudaGetLastError();
 }
 
 }  // namespace svdq

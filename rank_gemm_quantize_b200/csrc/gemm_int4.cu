@@ -75,6 +75,7 @@ struct SmemI4 {
   static constexpr int kTotal = kBarOff + ((kBarBytes + 127) / 128) * 128 + 1024;
 };
 static_assert(SmemI4::kTotal <= 232448, "shared memory budget");
+static_assert(kBN % kWeightBoxRows == 0 && kBM % kActBoxRows == 0, "operand tiles are whole boxes");
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_int4_kernel(const GemmParams p, const __grid_constant__ GemmMaps maps) {
@@ -98,7 +99,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_tiles = (p.M_pad / kBM) * n_blocks;
   const int n_groups = p.K / 64;
   const int n_main = p.K / kBK;
-  const int n_lr = p.TP / 32;  // branch k-tiles: every split partial of T
+  const int n_lr = p.RP / 32;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -161,13 +162,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* st = smem + s * L::kStage;
           if (k < n_main) {
             mbar_arrive_expect_tx(&full[s], L::kA + L::kB);
-            tma_load_2d(st, &maps.a, &full[s], k * kBK, m0);
-            tma_load_2d(st + L::kA, &maps.b, &full[s], k * kBK, n0);
+#pragma unroll
+            for (int h = 0; h < kBM / kActBoxRows; ++h)
+              tma_load_2d(st + h * kActBoxRows * kBK, &maps.a, &full[s], k * kBK, m0 + h * kActBoxRows);
+#pragma unroll
+            for (int h = 0; h < kBN / kWeightBoxRows; ++h)
+              tma_load_2d(st + L::kA + h * kWeightBoxRows * kBK, &maps.b, &full[s], k * kBK, n0 + h * kWeightBoxRows);
           } else {
             const int c = k - n_main;  // 32-column slice of the branch
             mbar_arrive_expect_tx(&full[s], kBM * 64 + kBN * 64);
             tma_load_2d(st, &maps.t, &full[s], c * 32, m0);
-            tma_load_2d(st + L::kA, &maps.l2, &full[s], (c % (p.RP / 32)) * 32, n0);
+#pragma unroll
+            for (int h = 0; h < kBN / kWeightBoxRows; ++h)
+              tma_load_2d(st + L::kA + h * kWeightBoxRows * 64, &maps.l2, &full[s], c * 32,
+                          n0 + h * kWeightBoxRows);
           }
         }
       }
@@ -340,7 +348,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-int gemm_int4_bn() { return kBN; }
 
 cudaError_t launch_gemm_int4(const GemmParams& p, const GemmMaps& maps, cudaStream_t stream) {
   static bool attr_set = false;

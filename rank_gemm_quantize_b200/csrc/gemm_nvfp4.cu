@@ -17,8 +17,7 @@
 //   warp 0  producer: for each tile, a bulk copy of the bias slice, then the
 //           k-tiles (A and B codes by TMA, their scale-factor atoms by bulk
 //           copy; four copies in flight per stage) followed by the branch
-//           k-tiles (a 32-column slice of one of the activation kernel's
-//           partials of T' and the matching slice of L2^T), through a 4-stage
+//           k-tiles (a 32-column slice of T' and of L2^T), through a 4-stage
 //           shared-memory ring;
 //   warp 1  TMEM owner and MMA issuer (one thread): scale factors to TMEM
 //           with tcgen05.cp, then 4 block-scaled MMAs per k-tile, 2 kind::f16
@@ -56,6 +55,7 @@ struct SmemNv {
   static constexpr int kTotal = kBarOff + 256 + 1024;
 };
 static_assert(SmemNv::kTotal <= 232448, "shared memory budget");
+static_assert(kBN % kWeightBoxRows == 0 && kBM % kActBoxRows == 0, "operand tiles are whole boxes");
 
 // TMEM columns: accumulator [0, 256), then one scale-factor slot per
 // shared-memory stage (A: 16 columns, B: 32), so copying the next k-tile's
@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_tiles = (p.M_pad / kBM) * n_blocks;
   const int kb_total = p.K / 64;
   const int n_main = (p.K + 255) / 256;
-  const int n_lr = p.TP / 32;  // branch k-tiles: every split partial of T
+  const int n_lr = p.RP / 32;
   const int n_items = n_main + n_lr;
 
   if (threadIdx.x == 0) {
@@ -143,8 +143,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int kb0 = k * 4;
             const int nkb = min(4, kb_total - kb0);
             mbar_arrive_expect_tx(&full[s], L::kA + L::kB + nkb * 512 * (1 + kBN / 128));
-            tma_load_2d(st, &maps.a, &full[s], k * kBKBytes, m0);
-            tma_load_2d(st + L::kA, &maps.b, &full[s], k * kBKBytes, n0);
+#pragma unroll
+            for (int h = 0; h < kBM / kActBoxRows; ++h)
+              tma_load_2d(st + h * kActBoxRows * kBKBytes, &maps.a, &full[s], k * kBKBytes, m0 + h * kActBoxRows);
+#pragma unroll
+            for (int h = 0; h < kBN / kWeightBoxRows; ++h)
+              tma_load_2d(st + L::kA + h * kWeightBoxRows * kBKBytes, &maps.b, &full[s], k * kBKBytes, n0 + h * kWeightBoxRows);
             const uint8_t* sa = reinterpret_cast<const uint8_t*>(p.sa) + (static_cast<size_t>(mb) * kb_total + kb0) * 512;
             bulk_load(st + L::kA + L::kB, sa, nkb * 512, &full[s]);
 #pragma unroll
@@ -157,7 +161,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int c = k - n_main;  // 32-column slice of the branch
             mbar_arrive_expect_tx(&full[s], kBM * 64 + kBN * 64);
             tma_load_2d(st, &maps.t, &full[s], c * 32, m0);
-            tma_load_2d(st + L::kA, &maps.l2, &full[s], (c % (p.RP / 32)) * 32, n0);
+#pragma unroll
+            for (int h = 0; h < kBN / kWeightBoxRows; ++h)
+              tma_load_2d(st + L::kA + h * kWeightBoxRows * 64, &maps.l2, &full[s], c * 32,
+                          n0 + h * kWeightBoxRows);
           }
         }
       }
@@ -288,7 +295,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-int gemm_nvfp4_bn() { return kBN; }
 
 cudaError_t launch_gemm_nvfp4(const GemmParams& p, const GemmMaps& maps, cudaStream_t stream) {
   static bool attr_set = false;

@@ -17,8 +17,10 @@ struct ActQuantParams {
   const __nv_bfloat16* L1T;  // [RP, K]: transposed, zero-padded down-projection factor
   uint8_t* codes;          // INT4: [M_pad, K] E4M3 bytes of the integer codes; NVFP4: [M_pad, K/2] packed E2M1
   void* scales;            // INT4: float [K/64][M_pad]; NVFP4: scale-factor atoms [M_pad/128][K/64][512]
-  __nv_bfloat16* T;        // [M_pad, TP] bf16: split partials of t_scale * (x_hat L1), RP columns each
-  int split, TP;           // K shares per 64-row block (from act_quant_split) and TP = split * RP
+  __nv_bfloat16* T;        // [M_pad, RP] bf16 = t_scale * (x_hat L1)
+  int split;               // K shares per 128-row block (from act_quant_split)
+  float* Tpart;            // [split][M_pad][RP] float partials over the K shares (split > 1)
+  int* counters;           // [M_pad / 128] arrival counts of the shares, zero between launches
   float g_x;               // NVFP4 activation tensor scale
   float denom;             // NVFP4: fp32(6 * g_x)
   float t_scale;           // 1 (INT4) or 1 / (g_x g_w) (NVFP4)
@@ -29,17 +31,15 @@ struct ActQuantMaps {
   CUtensorMap l1t;  // L1T [RP, K] bf16, box {64, RP}, 128-byte swizzle
 };
 int act_quant_box_rows();
-// K shares per 64-row block for M_pad rows: the grid fills the GPU in one wave.
+// K shares per 128-row block for M_pad rows: the grid fills the GPU in one wave.
 int act_quant_split(int M_pad, int K, int fmt, int rp, int sms);
+// Row blocks the per-layer arrival counters cover (M_pad / 128 at most this).
+constexpr int kMaxRowBlocks = 65536;
 cudaError_t launch_act_quant(const ActQuantParams& p, const ActQuantMaps& maps, int fmt, int rp, cudaStream_t stream);
-// out[m, c] = sum over the split partials of T (float), for introspection.
-cudaError_t launch_t_partials_sum(const __nv_bfloat16* Tp, int M_pad, int RP, int split, float* out,
-                                  cudaStream_t stream);
 
 // ---------------------------------------------------------------- GEMMs
 struct GemmParams {
   int M, N, K, RP;
-  int TP;                      // columns of T: the activation kernel's split partials, RP each
   __nv_bfloat16* Y;            // [M, N]
   const __nv_bfloat16* bias;   // [N_pad], zero beyond N
   const void* sa;              // activation scales (layout of ActQuantParams::scales)
@@ -51,11 +51,17 @@ struct GemmParams {
 struct GemmMaps {
   CUtensorMap a;   // activation codes
   CUtensorMap b;   // weight codes
-  CUtensorMap t;   // T [M_pad, TP] bf16 (partials; each is contracted with L2)
+  CUtensorMap t;   // T [M_pad, RP] bf16
   CUtensorMap l2;  // L2T [N_pad, RP] bf16
 };
-int gemm_nvfp4_bn();  // tile width (rows of the weight box) of each GEMM
-int gemm_int4_bn();
+// Rows of one TMA box of the weight codes, of L2^T and of the activation codes.
+// The GEMMs load a tile's operand rows as several boxes: copies in flight,
+// not their size, set the TMA throughput of an SM.
+constexpr int kWeightBoxRows = 128;
+#ifndef SVDQ_ACT_BOX_ROWS
+#define SVDQ_ACT_BOX_ROWS 128
+#endif
+constexpr int kActBoxRows = SVDQ_ACT_BOX_ROWS;
 cudaError_t launch_gemm_nvfp4(const GemmParams& p, const GemmMaps& maps, cudaStream_t stream);
 cudaError_t launch_gemm_int4(const GemmParams& p, const GemmMaps& maps, cudaStream_t stream);
 

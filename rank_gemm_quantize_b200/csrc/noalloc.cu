@@ -29,9 +29,9 @@ void set_last_error(const std::string& msg);
 namespace {
 
 // Largest workspace the array holds: enough for M x K = 4608 x 3072 in either
-// format at rank <= 32 (about 15.5 MiB for INT4, 8.4 MiB for NVFP4, with the
-// activation kernel's partials of T).
-constexpr size_t kScratchBytes = size_t(16) << 20;
+// format up to rank 128 (at rank 32: about 17 MiB for INT4, 10 MiB for
+// NVFP4, including the activation kernel's float partials of T).
+constexpr size_t kScratchBytes = size_t(32) << 20;
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mutex;

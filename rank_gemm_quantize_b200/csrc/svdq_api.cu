@@ -73,7 +73,6 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
 // Weight-side padding: every GEMM tile width divides it, so per-tile scale
 // copies never leave the buffers.
 constexpr int kNPad = 256;
-inline int gemm_bn(int fmt) { return fmt == SVDQ_INT4_G64 ? gemm_int4_bn() : gemm_nvfp4_bn(); }
 
 // Small cache of tensor maps keyed by (device pointer, rows): encoding a map
 // costs microseconds of host time, and callers usually cycle through a few
@@ -106,8 +105,8 @@ struct MapCache {
 
 struct WsLayout {
   int M_pad;
-  int split, TP;  // activation-kernel K shares and the width of T (split * RP)
-  size_t codes, scales, T, total;
+  int split;      // activation-kernel K shares per 128-row block
+  size_t codes, scales, T, Tpart, total;
 };
 
 }  // namespace
@@ -127,6 +126,7 @@ struct svdq_layer {
   uint8_t* wcodes = nullptr;     // INT4 [N_pad, K] E4M3 bytes; NVFP4 [N_pad, K/2]
   void* wscales = nullptr;       // INT4 float [K/64][N_pad]; NVFP4 atoms [N_pad/128][K/64][512]
   int* status = nullptr;         // device status word
+  int* k1_counters = nullptr;    // activation-kernel arrival counters per 128-row block (zero between launches)
   CUtensorMap map_b{}, map_l2{}, map_l1t{};
   MapCache<8> ws_maps;  // (workspace, M) -> activation codes map (a), T map (b)
   MapCache<8> x_maps;   // (X, M) -> X map (a)
@@ -144,9 +144,10 @@ WsLayout ws_layout(const svdq_layer* h, int M) {
   w.codes = 0;
   w.scales = align256(cbytes);
   w.split = act_quant_split(w.M_pad, h->K, h->fmt, h->RP, h->sms);
-  w.TP = w.split * h->RP;
   w.T = w.scales + align256(sbytes);
-  w.total = w.T + align256(static_cast<size_t>(w.M_pad) * w.TP * 2);
+  w.Tpart = w.T + align256(static_cast<size_t>(w.M_pad) * h->RP * 2);
+  const size_t part = w.split > 1 ? static_cast<size_t>(w.split) * w.M_pad * h->RP * 4 : 0;
+  w.total = w.Tpart + align256(part);
   return w;
 }
 
@@ -192,17 +193,18 @@ void free_layer(svdq_layer* h) {
   cudaFree(h->wcodes);
   cudaFree(h->wscales);
   cudaFree(h->status);
+  cudaFree(h->k1_counters);
   delete h;
 }
 
 svdq_status build_static_maps(svdq_layer* h) {
   const bool i4 = h->fmt == SVDQ_INT4_G64;
   const uint64_t row = i4 ? h->K : h->K / 2;
-  if (!make_map(&h->map_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, row, h->N_pad, row, 128, gemm_bn(h->fmt),
+  if (!make_map(&h->map_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, row, h->N_pad, row, 128, kWeightBoxRows,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (weight codes) failed");
   if (!make_map(&h->map_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->L2T, h->RP, h->N_pad, static_cast<uint64_t>(h->RP) * 2,
-                32, gemm_bn(h->fmt), CU_TENSOR_MAP_SWIZZLE_64B))
+                32, kWeightBoxRows, CU_TENSOR_MAP_SWIZZLE_64B))
     return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (L2) failed");
   if (!make_map(&h->map_l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->L1T, h->K, h->RP, static_cast<uint64_t>(h->K) * 2, 64,
                 h->RP, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -331,9 +333,10 @@ svdq_status start_prepare(const svdq_config* cfg, const void* W, const void* bia
     return s;
   };
   if ((e = dalloc(&h->s, K * 4)) || (e = dalloc(&h->inv_s, K * 4)) || (e = dalloc(&h->bias, h->N_pad * 2)) ||
-      (e = dalloc(&h->status, 16)))
+      (e = dalloc(&h->status, 16)) || (e = dalloc(&h->k1_counters, kMaxRowBlocks * sizeof(int))))
     return bail(e);
   cudaMemsetAsync(h->status, 0, 16, st);
+  cudaMemsetAsync(h->k1_counters, 0, kMaxRowBlocks * sizeof(int), st);
   cudaMemsetAsync(h->bias, 0, h->N_pad * 2, st);  // padded with zeros to the weight padding
   if (bias) cudaMemcpyAsync(h->bias, bias, N * 2, cudaMemcpyDeviceToDevice, st);
 
@@ -431,10 +434,12 @@ svdq_status svd_factors(svdq_layer* h, const float* W_hat, __nv_bfloat16* L1, __
 }
 
 svdq_status launch_k1(svdq_layer* h, const void* X, int M, uint8_t* codes, void* scales, __nv_bfloat16* T,
-                      const WsLayout& w, cudaStream_t st) {
+                      float* Tpart, const WsLayout& w, cudaStream_t st) {
+  if (w.M_pad / 128 > kMaxRowBlocks) return fail(SVDQ_ERR_INVALID_ARG, "M exceeds the supported row count");
   ActQuantParams p{};
   p.split = w.split;
-  p.TP = w.TP;
+  p.Tpart = Tpart;
+  p.counters = h->k1_counters;
   p.X = static_cast<const __nv_bfloat16*>(X);
   p.M = M;
   p.K = h->K;
@@ -556,7 +561,8 @@ svdq_status forward_impl(svdq_layer* h, const void* X, int M, void* Y, void* wor
   void* scales = base + w.scales;
   __nv_bfloat16* T = reinterpret_cast<__nv_bfloat16*>(base + w.T);
   if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[0]), st));
-  svdq_status e = launch_k1(h, X, M, codes, scales, T, w, st);
+  float* Tpart = reinterpret_cast<float*>(base + w.Tpart);
+  svdq_status e = launch_k1(h, X, M, codes, scales, T, Tpart, w, st);
   if (e) return e;
   if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[1]), st));
   auto* we = h->ws_maps.find(workspace, M);
@@ -564,9 +570,9 @@ svdq_status forward_impl(svdq_layer* h, const void* X, int M, void* Y, void* wor
     we = h->ws_maps.insert(workspace, M);
     const bool i4 = h->fmt == SVDQ_INT4_G64;
     const uint64_t row = i4 ? h->K : h->K / 2;
-    if (!make_map(&we->a, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, row, w.M_pad, row, 128, 128,
+    if (!make_map(&we->a, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, row, w.M_pad, row, 128, kActBoxRows,
                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&we->b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, w.TP, w.M_pad, static_cast<uint64_t>(w.TP) * 2, 32,
+        !make_map(&we->b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, h->RP, w.M_pad, static_cast<uint64_t>(h->RP) * 2, 32,
                   128, CU_TENSOR_MAP_SWIZZLE_64B)) {
       we->key = nullptr;
       return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (activations) failed");
@@ -577,7 +583,6 @@ svdq_status forward_impl(svdq_layer* h, const void* X, int M, void* Y, void* wor
   p.N = h->N;
   p.K = h->K;
   p.RP = h->RP;
-  p.TP = w.TP;
   p.Y = static_cast<__nv_bfloat16*>(Y);
   p.bias = h->bias;
   p.sa = scales;
@@ -620,16 +625,14 @@ svdq_status svdq_quantize_activations(svdq_layer_t h, const void* X, int M, void
     return fail(SVDQ_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const WsLayout w = ws_layout(h, M);
-  // the forward keeps T as split partials; this call returns their float sum
-  void* Tp = nullptr;
-  cudaError_t ce = cudaMallocAsync(&Tp, static_cast<size_t>(w.M_pad) * w.TP * 2, st);
-  if (ce != cudaSuccess) return fail(SVDQ_ERR_OOM, std::string("T partials: ") + cudaGetErrorString(ce));
-  svdq_status e = launch_k1(h, X, M, static_cast<uint8_t*>(codes), scales, static_cast<__nv_bfloat16*>(Tp), w, st);
-  if (e == SVDQ_OK) {
-    ce = launch_t_partials_sum(static_cast<const __nv_bfloat16*>(Tp), w.M_pad, h->RP, w.split, static_cast<float*>(T), st);
-    if (ce != cudaSuccess) e = fail(SVDQ_ERR_CUDA, std::string("T partial sum: ") + cudaGetErrorString(ce));
+  // float partials over the K shares: a scratch buffer of this call's own
+  float* Tpart = nullptr;
+  if (w.split > 1) {
+    cudaError_t ce = cudaMallocAsync(reinterpret_cast<void**>(&Tpart), w.total - w.Tpart, st);
+    if (ce != cudaSuccess) return fail(SVDQ_ERR_OOM, std::string("T partials: ") + cudaGetErrorString(ce));
   }
-  cudaFreeAsync(Tp, st);
+  svdq_status e = launch_k1(h, X, M, static_cast<uint8_t*>(codes), scales, static_cast<__nv_bfloat16*>(T), Tpart, w, st);
+  if (Tpart) cudaFreeAsync(Tpart, st);
   return e;
 }
 
