@@ -121,7 +121,10 @@ SVDQ_API svdq_status svdq_prepare_weights_with_factors(const svdq_config* cfg, c
                                               const float* act_absmax, const void* L1, const void* L2, void* stream,
                                               svdq_layer_t* out);
 
-/* Bytes of workspace svdq_linear_forward needs for M rows. */
+/* Bytes of workspace svdq_linear_forward needs for M rows: the activation
+ * codes and scales, T, and the activation kernel's float partials of T over
+ * its shares of K (their number depends on M, K, the rank and the device's SM
+ * count, so query this on the device the layer lives on). */
 SVDQ_API svdq_status svdq_workspace_size(svdq_layer_t layer, int M, size_t* bytes);
 
 /* The hot path: Y = Q(X diag(s)^-1) Q(R) + (X diag(s)^-1 L1) L2 + b, bf16 out.
@@ -131,7 +134,11 @@ SVDQ_API svdq_status svdq_workspace_size(svdq_layer_t layer, int M, size_t* byte
  *   X          device bf16 [M, K]
  *   Y          device bf16 [M, N] (overwritten)
  *   workspace  device buffer of at least svdq_workspace_size(layer, M) bytes,
- *              256-byte aligned; its contents need no initialisation. */
+ *              256-byte aligned; its contents need no initialisation.
+ * M_pad / 128 = ceil(M / 128) must not exceed 65536 (the layer keeps one
+ * arrival counter per 128-row block for the activation kernel; they return
+ * to zero at the end of every launch, which is why a layer serves one stream
+ * at a time). */
 SVDQ_API svdq_status svdq_linear_forward(svdq_layer_t layer, const void* X, int M, void* Y, void* workspace,
                                 size_t workspace_bytes, void* stream);
 
