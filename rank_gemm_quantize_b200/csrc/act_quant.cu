@@ -393,12 +393,11 @@ template <int FMT, int RP>
 cudaError_t launch_rp(const ActQuantParams& p, const ActQuantMaps& maps, cudaStream_t stream) {
   using S = K1Shape<RP>;
   auto kern = act_quant_kernel<FMT, RP>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  cudaError_t e = once_per_device(attr_done, [&] {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal);
+  });
+  if (e != cudaSuccess) return e;
   act_quant_kernel<FMT, RP><<<(p.M_pad / kRows) * p.split, kThreads, S::kTotal, stream>>>(p, maps);
   return cudaGetLastError();
 }

@@ -4,6 +4,7 @@
 // of the Blackwell tensor cores. All PTX here is hand-written inline assembly.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -13,6 +14,21 @@
 #include "svdq.h"
 
 namespace svdq {
+
+// Function attributes (the dynamic shared-memory size) live in each device's
+// context: run `set` once per device the process launches on.
+template <class Set>
+inline cudaError_t once_per_device(std::atomic<unsigned long long>& done, Set set) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return set();
+  const unsigned long long bit = 1ull << dev;
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = set();
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // Device status words (one int per launch, written only on failure).
 enum DeviceStatus : int {

@@ -350,14 +350,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 
 cudaError_t launch_gemm_int4(const GemmParams& p, const GemmMaps& maps, cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SmemI4::kTotal);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  cudaError_t e = once_per_device(attr_done, [] {
+    return cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SmemI4::kTotal);
+  });
+  if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   const int n_tiles = (p.M_pad / kBM) * ((p.N + kBN - 1) / kBN);

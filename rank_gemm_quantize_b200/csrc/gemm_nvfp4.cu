@@ -297,12 +297,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 
 cudaError_t launch_gemm_nvfp4(const GemmParams& p, const GemmMaps& maps, cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SmemNv::kTotal);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  cudaError_t e = once_per_device(attr_done, [] {
+    return cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SmemNv::kTotal);
+  });
+  if (e != cudaSuccess) return e;
   static int sms = 0;
   if (sms == 0) {
     int dev = 0;
