@@ -13,15 +13,20 @@
 // tensor scales and the bias and stores bf16 once.
 //
 // Persistent kernel, one CTA per SM, 128 x 256 output tiles taken round-robin.
-// Warp roles (10 warps):
+// Warp roles (11 warps):
 //   warp 0  producer: for each tile, a bulk copy of the bias slice, then the
 //           k-tiles (A and B codes by TMA, their scale-factor atoms by bulk
-//           copy; four copies in flight per stage) followed by the branch
-//           k-tiles (a 32-column slice of T' and of L2^T), through a 4-stage
-//           shared-memory ring;
-//   warp 1  TMEM owner and MMA issuer (one thread): scale factors to TMEM
-//           with tcgen05.cp, then 4 block-scaled MMAs per k-tile, 2 kind::f16
-//           MMAs per branch k-tile; commits release the stage / mark the tile;
+//           copy) followed by the branch k-tiles (a 32-column slice of T'
+//           and of L2^T), through a 4-stage shared-memory ring;
+//   warp 10 scale factors: copies each stage's scale-factor atoms into that
+//           stage's TMEM slot with tcgen05.cp and commits them to the stage's
+//           sf_ready barrier. Copies issued from the MMA thread serialise
+//           with its MMAs (about 47 cycles per copy, 12 per k-tile, against
+//           512 cycles of MMAs); from a thread of their own they overlap;
+//   warp 1  TMEM owner and MMA issuer (one thread): per k-tile, once the
+//           stage's scale factors are in TMEM, 4 block-scaled MMAs; per
+//           branch k-tile 2 kind::f16 MMAs; commits release the stage / mark
+//           the tile;
 //   warps 2-9 epilogue: each copies its 32 rows x 128 columns of the
 //           accumulator to registers and releases TMEM at once, so the next
 //           tile's MMAs overlap the scaling, bias and bf16 stores.
@@ -41,7 +46,8 @@ constexpr int kBN = 256;
 constexpr int kBKBytes = 128;  // 256 E2M1 values per row per k-tile
 constexpr int kStages = 4;
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = (2 + kEpiWarps) * 32;
+constexpr int kCpWarp = 2 + kEpiWarps;  // copies scale factors into TMEM
+constexpr int kThreads = (3 + kEpiWarps) * 32;
 
 struct SmemNv {
   static constexpr int kA = kBM * kBKBytes;   // 16 KB
@@ -78,7 +84,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bias_full = acc_empty + 1;   // [2]
   uint64_t* bias_empty = bias_full + 2;  // [2]
   uint64_t* drain = bias_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* sf_ready = drain + 1;        // [kStages] scale factors of the stage are in TMEM
+  uint64_t* cp_done = sf_ready + kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cp_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -102,6 +110,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bias_empty[b], kEpiWarps);
     }
     mbar_init(drain, 1);
+    for (int s = 0; s < kStages; ++s) mbar_init(&sf_ready[s], 1);
+    mbar_init(cp_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -189,7 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       for (int k = 0; k < n_items && ok; ++k, ++it) {
         const int s = it % kStages;
-        ok = mbar_wait(&full[s], (it / kStages) & 1, abort_flag, p.status);
+        ok = mbar_wait(&sf_ready[s], (it / kStages) & 1, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
         if (lane == 0) {  // one fixed thread issues every tcgen05 op, so its commits track them all
@@ -200,15 +210,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nkb = min(4, kb_total - k * 4);
             const uint32_t t_sfa = tmem + kSfaCol + s * kSfSlotCols;
             const uint32_t t_sfb = tmem + kSfbCol + s * kSfSlotCols;
-            const uint32_t sfa_base = smem_u32(st + L::kA + L::kB);
-            const uint32_t sfb_base = sfa_base + L::kSfa;
-            for (int j = 0; j < nkb; ++j) {
-              tmem_cp_32x128b_x4(t_sfa + 4 * j, smem_desc(sfa_base + 512 * j, 16, 128, kSwNone));
-#pragma unroll
-              for (int h = 0; h < kBN / 128; ++h)
-                tmem_cp_32x128b_x4(t_sfb + (kBN / 32) * j + 4 * h,
-                                   smem_desc(sfb_base + h * 2048 + 512 * j, 16, 128, kSwNone));
-            }
             for (int j = 0; j < nkb; ++j) {
               const uint64_t ad = smem_desc(a_base + 32 * j, 16, 1024, kSw128);
               const uint64_t bd = smem_desc(b_base + 32 * j, 16, 1024, kSw128);
@@ -228,6 +229,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
       }
     }
+  } else if (warp == kCpWarp) {
+    // ------------------------------------------------------------ scale factors to TMEM
+    // One stage ahead of the MMA thread at most (it waits for each stage's
+    // copies): the copies and the MMAs come from different threads.
+    if (lane == 0) {
+      bool ok = true;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+        for (int k = 0; k < n_items && ok; ++k, ++it) {
+          const int s = it % kStages;
+          ok = mbar_wait(&full[s], (it / kStages) & 1, abort_flag, p.status);
+          if (!ok) break;
+          tc_fence_after();
+          if (k < n_main) {
+            uint8_t* st = smem + s * L::kStage;
+            const int nkb = min(4, kb_total - k * 4);
+            const uint32_t t_sfa = tmem + kSfaCol + s * kSfSlotCols;
+            const uint32_t t_sfb = tmem + kSfbCol + s * kSfSlotCols;
+            const uint32_t sfa_base = smem_u32(st + L::kA + L::kB);
+            const uint32_t sfb_base = sfa_base + L::kSfa;
+            for (int j = 0; j < nkb; ++j) {
+              tmem_cp_32x128b_x4(t_sfa + 4 * j, smem_desc(sfa_base + 512 * j, 16, 128, kSwNone));
+#pragma unroll
+              for (int h = 0; h < kBN / 128; ++h)
+                tmem_cp_32x128b_x4(t_sfb + (kBN / 32) * j + 4 * h,
+                                   smem_desc(sfb_base + h * 2048 + 512 * j, 16, 128, kSwNone));
+            }
+          }
+          tc_commit(&sf_ready[s]);
+        }
+      }
+      tc_commit(cp_done);  // arrives once every copy issued above has finished
+      volatile int no_abort = 0;
+      mbar_wait(cp_done, 0, &no_abort, nullptr);
+    }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
     const int ew = warp - 2;                  // 0..7
