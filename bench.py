@@ -1,13 +1,14 @@
 #!/usr/bin/env python
 """Benchmark of the SVDQuant W4A4 + low-rank linear layer on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 1]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 3]
 
 One step = one pass of the whole hot path (svdq_linear_forward: the activation
 kernel + the 4-bit GEMM with the fused low-rank/bias epilogue) over one batch
 of the configuration's synthetic inputs (for the MLP-pair configurations, both
-layers). Default workload: the FLUX-like attention projection (X [4608, 3072]
-bf16, W [3072, 3072], rank 32, INT4 group 64). Prints one JSON line on rank 0.
+layers). Default workload: the FLUX-like MLP pair in NVFP4 (up 4608 x 3072 ->
+12288, then down 4608 x 12288 -> 3072, rank 32, E2M1 group 16), the largest
+configuration. Prints one JSON line on rank 0.
 
 Multi-GPU (torchrun, one process per GPU): the layer is token-parallel - every
 rank runs its own batch against its own copy of the weights, with no
@@ -84,6 +85,52 @@ def load_layers(args):
         kw["fmt"] = args.fmt
     layers = workloads.config(args.config, **kw)
     return layers
+
+
+# A timed region shorter than this is a burst: the clocks have not settled
+# under the power cap, so the burst peak is the fair denominator.
+BURST_REGION_S = 1.0
+
+
+def tensor_peak_for(peaks: dict, fmt: str, timed_region_s: float):
+    """(peak TFLOP/s, description): the measured bf16 GEMM peak for the length
+    of the timed region (burst when it is shorter than BURST_REGION_S, else
+    sustained) times the nominal rate ratio of the MMA kind the format uses."""
+    burst = timed_region_s < BURST_REGION_S
+    key = "bf16_tflops" if burst else "bf16_tflops_sustained"
+    kind = "mxf4nvf4" if fmt == "nvfp4_g16" else "f8f6f4"
+    desc = (f"bf16 {'burst' if burst else 'sustained'} {peaks[key]} TFLOP/s x {RATE_VS_BF16[fmt]:g} "
+            f"(nominal {kind}/bf16 rate; timed region {timed_region_s:.3f} s)")
+    return peaks[key] * RATE_VS_BF16[fmt], desc
+
+
+def ws_bytes_lower_bound(L) -> int:
+    """Activation codes + scales + T of one forward (the K-share partials left out)."""
+    M_pad = (L.M + 127) // 128 * 128
+    codes = M_pad * L.K if L.fmt == "int4_g64" else M_pad * L.K // 2
+    scales = M_pad * (L.K // 64) * 4 if L.fmt == "int4_g64" else M_pad * (L.K // 16)
+    return codes + scales + M_pad * ((L.rank + 31) // 32 * 32) * 2
+
+
+def rotation_sets(layers) -> tuple[int, int]:
+    """(sets, bytes per set): enough rotating copies of inputs, outputs,
+    workspace and prepared weights that one step's data is out of L2 again
+    when its set comes back."""
+    set_bytes = 0
+    for L in layers:
+        set_bytes += L.M * L.K * 2 + L.M * L.N * 2 + ws_bytes_lower_bound(L)
+        set_bytes += L.N * L.K // 2 * (2 if L.fmt == "int4_g64" else 1) + L.N * L.K // 16
+    return max(2, math.ceil(2 * L2_BYTES / max(set_bytes, 1))), set_bytes
+
+
+def config_dict(args, layers) -> dict:
+    """The `config` object of the JSON line, identical in both arms."""
+    n_sets, set_bytes = rotation_sets(layers)
+    L = layers[0]
+    return {"workload": workload_desc(args.config, layers), "config_id": args.config,
+            "M": L.M, "K": L.K, "N": L.N, "rank": L.rank, "format": L.fmt, "layers_per_step": len(layers),
+            "l2": f"inputs larger than L2: {n_sets} rotating sets of prepared layer + X/Y/workspace "
+                  f"(>= {n_sets * set_bytes / 2**20:.0f} MiB > 2 x 126 MiB L2)"}
 
 
 def read_peaks():
@@ -236,11 +283,7 @@ def run_ours(args):
         g0 = rq.Layer.prepare(L.W.to(dev), L.bias.to(dev), a, L.fmt, L.rank, alpha=L.alpha)
         ex = g0.export()
         preps.append((L, X0, a, g0, ex))
-    set_bytes = 0
-    for (L, X0, a, g0, ex) in preps:
-        set_bytes += L.M * L.K * 2 + L.M * L.N * 2 + g0.workspace_size(L.M)
-        set_bytes += L.N * L.K // 2 * (2 if L.fmt == "int4_g64" else 1) + L.N * L.K // 16
-    n_sets = max(2, math.ceil(2 * L2_BYTES / max(set_bytes, 1)))
+    n_sets, _ = rotation_sets(layers)
     sets = []
     for s in range(n_sets):
         items = []
@@ -304,32 +347,98 @@ def run_ours(args):
     value = whole_job_tops(step_ops, K_steps, world, max_ms)
     ms_per_step = max_ms / K_steps
 
-    # ---- e2e through the public API with host buffers: H2D of X, forward, D2H of Y
+    # ---- e2e through the public API with host buffers. Every step copies its
+    # inputs in from pinned host memory and its outputs back out. The batches
+    # are independent, so step i+1's inputs travel host->device on one copy
+    # stream and step i-1's outputs device->host on another (PCIe is full
+    # duplex) while step i computes; events keep each rotating set's buffers
+    # from being overwritten before the step that last used them is done.
     e2e_steps = max(3, min(args.e2e_steps, K_steps))
     hostX = [L.X.pin_memory() for L in layers]
     hostY = [torch.empty(L.M, L.N, dtype=torch.bfloat16).pin_memory() for L in layers]
     h2d = sum(L.M * L.K * 2 for L in layers)
     d2h = sum(L.M * L.N * 2 for L in layers)
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
 
-    def e2e_step(i):
-        for li, (g, X, Y, ws) in enumerate(sets[i % n_sets]):
-            X.copy_(hostX[li], non_blocking=True)
-            g.forward(X, out=Y, workspace=ws)
-            hostY[li].copy_(Y, non_blocking=True)
+    def e2e_run(n):
+        fwd_done = [None] * n_sets  # forward of the last step that used the set (its X is free after it)
+        out_done = [None] * n_sets  # D2H of the last step that used the set (its Y is free after it)
+        for i in range(n):
+            k = i % n_sets
+            with torch.cuda.stream(s_in):
+                if fwd_done[k] is not None:
+                    s_in.wait_event(fwd_done[k])
+                for li, (g, X, Y, ws) in enumerate(sets[k]):
+                    X.copy_(hostX[li], non_blocking=True)
+                ev_in = torch.cuda.Event()
+                ev_in.record(s_in)
+            comp.wait_event(ev_in)
+            if out_done[k] is not None:
+                comp.wait_event(out_done[k])
+            for li, (g, X, Y, ws) in enumerate(sets[k]):
+                g.forward(X, out=Y, workspace=ws, stream=comp)
+            fwd_done[k] = torch.cuda.Event()
+            fwd_done[k].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(fwd_done[k])
+                for li, (g, X, Y, ws) in enumerate(sets[k]):
+                    hostY[li].copy_(Y, non_blocking=True)
+                out_done[k] = torch.cuda.Event()
+                out_done[k].record(s_out)
+        for ev in out_done:  # the region ends when the last output is on the host
+            if ev is not None:
+                comp.wait_event(ev)
 
-    for i in range(2):
-        e2e_step(i)
+    e2e_run(2)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(e2e_steps):
-        e2e_step(i)
-    e1.record()
+    e0.record(comp)
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
+    e2e_run(e2e_steps)
+    e1.record(comp)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e_value = whole_job_tops(step_ops, e2e_steps, world, e2e_ms)
+    # the last step's outputs reached the host: compare them with the device copies
+    for li, (g, X, Y, ws) in enumerate(sets[(e2e_steps - 1) % n_sets]):
+        if not torch.equal(hostY[li], Y.cpu()):
+            raise SystemExit("e2e: the host copy of the output differs from the device result")
+
+    # ---- the 4-bit weight-only (W4A16) baseline of the abstract's speedup
+    # claim, on the same workload: its own quantized weights per rotating
+    # set, the same X, timed the same way (outside the timed region above)
+    w4a16 = None
+    if not args.no_w4a16:
+        w4_sets = [[rq.WeightOnlyLayer(L.W.to(dev), L.bias.to(dev)) for L in layers] for _ in range(n_sets)]
+
+        def w4_step(i):
+            for li, (g, X, Y, ws) in enumerate(sets[i % n_sets]):
+                w4_sets[i % n_sets][li].forward(X, out=Y)
+
+        for i in range(max(3, W_steps)):
+            w4_step(i)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        w0.record()
+        for i in range(K_steps):
+            w4_step(i)
+        w1.record()
+        torch.cuda.synchronize()
+        w4_ms = max_over_ranks(w0.elapsed_time(w1), world, dev) / K_steps
+        w4_ops = sum(2.0 * L.M * L.K * L.N for L in layers)
+        w4a16 = {"ms_per_step": w4_ms, "tops": w4_ops / (w4_ms * 1e-3) / 1e12,
+                 "w4a4_speedup": w4_ms / ms_per_step,
+                 "what": "INT4 g64 weights alone (no smoothing, no branch), bf16 activations, tcgen05 kind::f16 "
+                         "after on-chip dequantization; one kernel per layer"}
+        for row in w4_sets:
+            for wl in row:
+                wl.close()
 
     # device status: no kernel gave up a wait
     for items in sets:
@@ -347,14 +456,13 @@ def run_ours(args):
     wl_key = f"cfg{args.config}_M{layers[0].M}_r{layers[0].rank}_{fmt}"
     g_ops = sum(gemm_ops(L.M, L.K, L.N, L.rank) for L in layers)
     g_s = sum(gemm_ms) * 1e-3
-    tensor_peak = peaks["bf16_tflops_sustained"] * RATE_VS_BF16[fmt]
+    tensor_peak, peak_desc = tensor_peak_for(peaks, fmt, elapsed_ms * 1e-3)
     gemm_name = "gemm_int4_kernel" if fmt == "int4_g64" else "gemm_nvfp4_kernel"
     traffic = traffic_for(gemm_name, wl_key)
     roofline = {"bound": "tensor", "kernel": gemm_name, "achieved": g_ops / g_s / 1e12,
                 "peak": tensor_peak, "unit": "TFLOP/s", "frac": g_ops / g_s / 1e12 / tensor_peak,
                 "traffic": traffic,
-                "peak_source": (f"{peak_kind} bf16 sustained {peaks['bf16_tflops_sustained']} TFLOP/s x "
-                                f"{RATE_VS_BF16[fmt]:g} (nominal {'mxf4nvf4' if fmt == 'nvfp4_g16' else 'f8f6f4'}/bf16 rate)"),
+                "peak_source": f"{peak_kind} {peak_desc}",
                 "algorithmic": "2MKN + 2MrN per launch", "frac_of_datasheet_dense": g_ops / g_s / 1e12 / DATASHEET_TOPS[fmt]}
     k_bytes = sum(k1_bytes(L.M, L.K, L.rank, fmt) for L in layers)
     k_s = sum(k1_ms) * 1e-3
@@ -381,11 +489,7 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "int4" if fmt == "int4_g64" else "nvfp4",
         "data": "synthetic",
-        "config": {"workload": workload_desc(args.config, layers), "config_id": args.config,
-                   "M": layers[0].M, "K": layers[0].K, "N": layers[0].N, "rank": layers[0].rank, "format": fmt,
-                   "layers_per_step": n_layers,
-                   "l2": f"inputs larger than L2: {n_sets} rotating sets of prepared layer + X/Y/workspace "
-                         f"({n_sets * set_bytes / 2**20:.0f} MiB > 2 x 126 MiB L2)"},
+        "config": config_dict(args, layers),
         "pct_of_datasheet_dense_peak": 100.0 * value / DATASHEET_TOPS[fmt],
         "roofline": roofline,
         "kernels": {"act_quant": {"ms": k1_ms, **k1_roof}, "gemm": {"ms": gemm_ms}},
@@ -393,12 +497,69 @@ def run_ours(args):
         "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps},
         "gpu_launches": 2 * n_layers * K_steps,
+        "w4a16_baseline": w4a16,
         "clocks": clocks,
         "impl": "ours",
     }
     print(json.dumps(out), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+# The method's ablations (msModelSlim SVDQuant entry, related terms: SmoothQuant
+# is the rank-0 special case; section 2.3 eq. 2: alpha sets the migration
+# strength): (name, rank, alpha, smooth).
+ABLATIONS = [
+    ("W4A4, no smoothing, no branch", 0, 0.5, False),
+    ("smoothing only (SmoothQuant, rank 0)", 0, 0.5, True),
+    ("low-rank branch without smoothing", None, 0.5, False),
+    ("SVDQuant alpha 0.3", None, 0.3, True),
+    ("SVDQuant alpha 0.5", None, 0.5, True),
+    ("SVDQuant alpha 0.7", None, 0.7, True),
+]
+
+
+def run_ablation(args):
+    """One JSON line: for each ablation of the method, the layer's normwise
+    error against the unquantized X W + b (float64) and its time per layer,
+    on the configuration's first layer, both formats."""
+    import torch
+
+    import rank_gemm_quantize_b200 as rq
+    import workloads
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    L = load_layers(args)[0]
+    X, W, b = L.X.to(dev), L.W.to(dev), L.bias.to(dev)
+    ref = X.double() @ W.double() + b.double()  # the layer without quantization
+    a = rq.calibrate_absmax(X)
+    rows = []
+    for fmt in workloads.FORMATS:
+        for name, rank, alpha, smooth in ABLATIONS:
+            r = L.rank if rank is None else rank
+            g = rq.Layer.prepare(W, b, a, fmt, r, alpha=alpha, smooth=smooth)
+            try:
+                Y = g.forward(X)
+                err = float(torch.linalg.norm(Y.double() - ref) / torch.linalg.norm(ref))
+                ws = g.workspace(L.M)
+                for _ in range(3):
+                    g.forward(X, out=Y, workspace=ws)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                n = 20
+                e0.record()
+                for _ in range(n):
+                    g.forward(X, out=Y, workspace=ws)
+                e1.record()
+                torch.cuda.synchronize()
+                us = e0.elapsed_time(e1) * 1e3 / n
+                rows.append({"format": fmt, "variant": name, "rank": r, "alpha": alpha, "smooth": smooth,
+                             "rel_err_vs_xw_plus_b": err, "us_per_layer": us,
+                             "tops": layer_ops(L.M, L.K, L.N, r) / (us * 1e-6) / 1e12})
+            finally:
+                g.close()
+    print(json.dumps({"ablation": rows, "config": config_dict(args, [L]) | {"layers_per_step": 1},
+                      "note": "L2-hot back-to-back timing of one layer; errors are normwise against float64 X W + b"}),
+          flush=True)
 
 
 def _blas_threads() -> int:
@@ -425,12 +586,23 @@ def _oracle_prepare(layers):
     return out
 
 
+def _rows_for(preps, seconds: float, M: int) -> int:
+    """Rows of the oracle's forward (row-local, so any row sample is a fair
+    sample of the batch) that take about `seconds` on this host."""
+    from oracle import svdquant as S
+    t = time.perf_counter()
+    for (L, X, p) in preps:
+        S.forward(p, X[:128])
+    per_row = max((time.perf_counter() - t) / 128, 1e-6)
+    return int(max(1, min(M, seconds / per_row)))
+
+
 def cpu_baseline(layers, budget_s: float = 10.0, rows=None):
     """The oracle's forward timed on the host cores on a row sample of the workload."""
     from oracle import svdquant as S
     preps = _oracle_prepare(layers)
     M = layers[0].M
-    r = rows or M
+    r = rows or _rows_for(preps, budget_s / 3, M)
     t_total, n, ops = 0.0, 0, 0.0
     while True:
         t = time.perf_counter()
@@ -453,13 +625,8 @@ def run_reference(args):
     layers = load_layers(args)
     from oracle import svdquant as S
     preps = _oracle_prepare(layers)
-    # size the row sample so that warmup + steps fit in ~2 minutes
-    t = time.perf_counter()
-    for (L, X, p) in preps:
-        S.forward(p, X[:64])
-    per_row = max((time.perf_counter() - t) / 64, 1e-6)
-    budget = 120.0 / max(1, args.steps + args.warmup)
-    rows = int(max(1, min(layers[0].M, budget / per_row)))
+    # size the row sample so that warmup + steps fit in about 80 s
+    rows = _rows_for(preps, 80.0 / max(1, args.steps + args.warmup), layers[0].M)
     for _ in range(args.warmup):
         for (L, X, p) in preps:
             S.forward(p, X[:rows])
@@ -477,9 +644,7 @@ def run_reference(args):
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": workload_desc(args.config, layers), "config_id": args.config, "M": layers[0].M,
-                   "K": layers[0].K, "N": layers[0].N, "rank": layers[0].rank, "format": fmt,
-                   "layers_per_step": len(layers)},
+        "config": config_dict(args, layers),
         "impl": "reference",
         "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -487,23 +652,32 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
-def main():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--config", type=int, default=3)
     ap.add_argument("--M", type=int, default=0)
     ap.add_argument("--rank", type=int, default=0)
     ap.add_argument("--fmt", choices=["int4_g64", "nvfp4_g16"], default=None)
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-w4a16", action="store_true", help="skip timing the weight-only baseline")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    args = ap.parse_args()
+    ap.add_argument("--ablation", action="store_true",
+                    help="print the error / time table of the method's ablations instead of the benchmark line")
+    return ap.parse_args(argv)
+
+
+def main():
+    args = parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.ablation:
+        run_ablation(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

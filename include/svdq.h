@@ -26,15 +26,22 @@
  *    svdq_quantize_activations never synchronize the host. A handle is used by
  *    one stream at a time; svdq_attach_lora must be stream-ordered with the
  *    forwards that precede it.
+ *  - Devices: a layer lives on the device that was current when it was
+ *    prepared. Calls that launch work on a layer (forward, quantize
+ *    activations, attach) must be made with that device current; otherwise
+ *    they return SVDQ_ERR_INVALID_ARG and launch nothing.
  *  - Errors: every call returns an svdq_status and never aborts or throws.
+ *    Argument errors (shapes, NULL or misaligned pointers, sizes) are
+ *    reported before any device work is queued.
  *    svdq_last_error() returns a thread-local description of the last failure.
  *    Launch failures come back as SVDQ_ERR_CUDA. A pipeline wait inside a
  *    kernel that gives up (it never blocks forever) is reported by
  *    svdq_device_status() as SVDQ_ERR_DEVICE_TIMEOUT.
  *  - Shape limits: K a multiple of 128; N a multiple of 16; M >= 1;
- *    1 <= rank (after any LoRA concatenation) <= 256 (section 2.6 recommends
+ *    0 <= rank (after any LoRA concatenation) <= 256 (section 2.6 recommends
  *    rank <= 128; the larger limit leaves room for LoRA adapters); only 2-D
- *    linear weights (section 2.6).
+ *    linear weights (section 2.6). Rank 0 is the smoothing-only special case
+ *    the entry's related terms name (SmoothQuant): no branch, R = diag(s) W.
  */
 #ifndef SVDQ_H_
 #define SVDQ_H_
@@ -67,25 +74,39 @@ typedef enum {
   SVDQ_NVFP4_G16 = 1  /* E2M1 values, 16 per group along K, E4M3 group scale, fp32 tensor scale */
 } svdq_format;
 
+/* svdq_config.flags */
+enum {
+  SVDQ_NO_SMOOTHING = 1  /* s = 1 for every channel (no migration; an ablation of eq. 1-2) */
+};
+
 typedef struct {
   int K;            /* input features (rows of W) */
   int N;            /* output features (columns of W) */
-  int rank;         /* r of the truncated SVD, 1..256 */
+  int rank;         /* r of the truncated SVD, 0..256 (0: no low-rank branch) */
   float alpha;      /* migration strength of eq. 2, in [0, 1] */
   float s_min;      /* lower clamp of s in eq. 2 (> 0; 1e-5 is the documented default) */
   svdq_format fmt;  /* 4-bit format of Q(.) */
+  unsigned int flags; /* 0, or SVDQ_NO_SMOOTHING */
 } svdq_config;
+
+/* LoRA adapter slots a layer holds at once. */
+#define SVDQ_MAX_ADAPTERS 8
 
 typedef struct svdq_layer* svdq_layer_t;
 
 typedef struct {
   int K, N, rank;   /* rank includes attached LoRA adapters */
-  int rank_pad;     /* rank rounded up to a multiple of 32 (layout of the branch buffers) */
+  int rank_pad;     /* rank rounded up to a multiple of 32 (layout of the branch buffers; 0 when rank is 0) */
   int fmt;          /* svdq_format */
   float alpha;
   float g_x;        /* NVFP4 static activation tensor scale (1 for INT4) */
   float g_w;        /* NVFP4 residual tensor scale (1 for INT4) */
   float t_scale;    /* factor applied to T before its bf16 store: 1 (INT4) or 1/(g_x g_w) (NVFP4) */
+  int base_rank;    /* rank of the SVD factors alone */
+  unsigned int flags;          /* svdq_config.flags of the layer */
+  unsigned int adapter_slots;  /* bit a set: adapter slot a holds an adapter */
+  int adapter_col_start[SVDQ_MAX_ADAPTERS + 1]; /* slot a owns branch columns [start[a], start[a+1]);
+                                                   the base factors own [0, start[0]) */
 } svdq_layer_info;
 
 /* Activation statistic A_scale of eq. 2 (section 2.3: per-channel absolute
@@ -166,12 +187,34 @@ SVDQ_API svdq_status svdq_linear_forward_noalloc(svdq_layer_t layer, const void*
 
 /* Attaches a LoRA adapter Y += scale X A B to the low-rank branch without
  * re-quantizing R (abstract: off-the-shelf LoRAs without re-quantization).
- * The branch sees X diag(s)^-1, so L1' = [L1 | bf16(diag(s) A)] and
- * L2' = [L2 ; bf16(scale B)]. The residual codes and scales are untouched.
- * Adapters accumulate: each call appends r_l more columns.
- *   A  device bf16 [K, r_l];  B  device bf16 [r_l, N];  1 <= rank + r_l <= 256.
- * Synchronizes `stream` before freeing the previous branch buffers. */
-SVDQ_API svdq_status svdq_attach_lora(svdq_layer_t layer, const void* A, const void* B, int r_l, float scale, void* stream);
+ * The branch sees X diag(s)^-1, so the adapter enters as the column block
+ * [bf16(diag(s) A)] of L1' and the row block [bf16(scale B)] of L2'. The
+ * residual codes and scales are untouched.
+ * The adapter takes the lowest free of SVDQ_MAX_ADAPTERS slots, returned in
+ * *slot_out (may be NULL). The branch is L1' = [L1 | F_a | F_b | ...],
+ * L2' = [L2 ; G_a ; G_b ; ...] with the occupied slots in slot order, so by
+ * default every adapter applies to every row (they accumulate); see
+ * svdq_linear_forward_masked for per-row selection.
+ *   A  device bf16 [K, r_l];  B  device bf16 [r_l, N];  rank + r_l <= 256.
+ * On any failure the layer is unchanged and *slot_out is -1. Synchronizes
+ * `stream` before freeing the previous branch buffers. */
+SVDQ_API svdq_status svdq_attach_lora(svdq_layer_t layer, const void* A, const void* B, int r_l, float scale, void* stream,
+                                      int* slot_out);
+
+/* Removes the adapter in `slot`: the branch buffers become byte for byte what
+ * they would be had the adapter never been attached (the remaining blocks are
+ * re-laid out in slot order), and the residual is untouched. Returns
+ * SVDQ_ERR_INVALID_ARG for an empty slot. Synchronizes `stream`. */
+SVDQ_API svdq_status svdq_detach_lora(svdq_layer_t layer, int slot, void* stream);
+
+/* svdq_linear_forward with per-row adapter selection (several requests with
+ * different LoRAs in one batch): row m of X uses the base branch plus the
+ * adapters whose slot bits are set in row_adapter_mask[m]; the branch columns
+ * of the other adapters are zeroed in T for that row before the GEMM, so a
+ * row gives exactly what a layer holding only its selected adapters would.
+ *   row_adapter_mask  device uint32 [M], 4-byte aligned (bit a = slot a). */
+SVDQ_API svdq_status svdq_linear_forward_masked(svdq_layer_t layer, const void* X, int M, void* Y, void* workspace,
+                                                size_t workspace_bytes, const uint32_t* row_adapter_mask, void* stream);
 
 /* The first kernel of the forward alone, into caller buffers, for inspection:
  *   codes   INT4: uint8 [M_pad, K], the E4M3 encoding of each integer code
@@ -181,10 +224,11 @@ SVDQ_API svdq_status svdq_attach_lora(svdq_layer_t layer, const void* A, const v
  *           NVFP4: uint8 E4M3 in 512-byte atoms, atom (m/128)*(K/64) + k/64,
  *                  byte (m%32)*16 + ((m/32)%4)*4 + (k/16)%4.
  *   T       bf16 [M_pad, rank_pad] = t_scale * (x_hat L1) (columns >= rank are 0)
- * The activation kernel splits K into shares whose float partial products it
- * sums in share order; this call allocates their scratch buffer on `stream`
- * and frees it before returning (the forward keeps it in its workspace).
- * with M_pad = M rounded up to a multiple of 128 (rows >= M are zero codes). */
+ * with M_pad = M rounded up to a multiple of 128 (rows >= M are zero codes).
+ * This call allocates: the activation kernel splits K into shares whose float
+ * partial products it sums in share order, and their scratch buffer is taken
+ * with cudaMallocAsync on `stream` and freed (cudaFreeAsync) before the call
+ * returns. The forward keeps that buffer in its workspace instead. */
 SVDQ_API svdq_status svdq_quantize_activations(svdq_layer_t layer, const void* X, int M, void* codes, void* scales, void* T,
                                       void* stream);
 
@@ -221,6 +265,35 @@ SVDQ_API svdq_status svdq_destroy(svdq_layer_t layer);
 
 /* Thread-local message of the last failed call ("" if none). */
 SVDQ_API const char* svdq_last_error(void);
+
+/* ------------------------------------------------------------------------
+ * The 4-bit weight-only baseline (W4A16) the SVDQuant abstract measures its
+ * 3.0x speedup against. W is quantized alone (no smoothing, no low-rank
+ * branch) with the same symmetric INT4 group-64 quantizer (scale = amax / 7
+ * per output column and 64 consecutive k); activations stay bf16:
+ *   Y = X bf16(fp32(q * scale))^T + b, fp32 accumulation, bf16 out.
+ * The packed codes stay 4-bit in device memory and are dequantized on chip in
+ * every forward. Same shape limits as the W4A4 layer (K % 128 == 0,
+ * N % 16 == 0), same error conventions. */
+typedef struct svdq_w4a16* svdq_w4a16_t;
+
+/* W device bf16 [K, N]; bias device bf16 [N] or NULL. Synchronizes `stream`. */
+SVDQ_API svdq_status svdq_w4a16_prepare(const void* W, const void* bias, int K, int N, void* stream,
+                                        svdq_w4a16_t* out);
+/* X device bf16 [M, K] -> Y device bf16 [M, N], one kernel on `stream`. */
+SVDQ_API svdq_status svdq_w4a16_forward(svdq_w4a16_t layer, const void* X, int M, void* Y, void* stream);
+/* The quantized weights, for inspection: codes host uint8 [N, K/2] (two's-
+ * complement nibbles, element 2j in bits 3:0), scales host float [K/64, N].
+ * Synchronizes `stream`. */
+SVDQ_API svdq_status svdq_w4a16_export(svdq_w4a16_t layer, void* codes, void* scales, void* stream);
+/* Frees the layer (synchronizes the device first). */
+SVDQ_API svdq_status svdq_w4a16_destroy(svdq_w4a16_t layer);
+
+/* Test hook for failure detection: the library's device allocation number
+ * `index` (0 = the next one) fails with SVDQ_ERR_OOM as if the device were out
+ * of memory, so that tests can check that every allocating call unwinds
+ * cleanly (no leak, no handle). A negative index switches the hook off. */
+SVDQ_API void svdq_debug_fail_allocation(long long index);
 
 /* Failure-detection self-test: launches a kernel that waits on a barrier no
  * one arrives on, with the library's bounded wait shortened to limit_ns, and

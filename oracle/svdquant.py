@@ -68,14 +68,18 @@ def weight_absmax(W: np.ndarray) -> np.ndarray:
     return np.max(np.abs(np.asarray(W, dtype=np.float64)), axis=1).astype(F32)
 
 
-def smoothing_factors(a: np.ndarray, w: np.ndarray, alpha: float, s_min: float = float(S_MIN)):
+def smoothing_factors(a: np.ndarray, w: np.ndarray, alpha: float, s_min: float = float(S_MIN), smooth: bool = True):
     """Eq. 2 of section 2.3: s = A_scale^alpha / W_scale^(1 - alpha), s >= s_min.
 
     Computed in float64 (sqrt(a) / sqrt(w) when alpha = 0.5, which is exact
     up to one rounding per operation), rounded once to float32, clamped below
     at s_min; a channel whose activation or weight statistic is 0 keeps s = 1.
-    inv_s = 1 / s in float32.
+    inv_s = 1 / s in float32. With smooth=False (the ablation without
+    migration) s = 1 for every channel.
     """
+    if not smooth:
+        ones = np.ones(np.asarray(a).shape, dtype=F32)
+        return ones, ones.copy()
     alpha = float(F32(alpha))  # alpha is a float32 parameter of the layer
     a64 = np.asarray(a, dtype=np.float64)
     w64 = np.asarray(w, dtype=np.float64)
@@ -149,13 +153,14 @@ def static_activation_scale(a: np.ndarray, inv_s: np.ndarray) -> np.float32:
 
 
 def prepare_from_factors(W, bias, act_absmax, fmt: str, alpha: float, L1, L2, sigma=None,
-                         s_min: float = float(S_MIN)) -> Prepared:
+                         s_min: float = float(S_MIN), smooth: bool = True) -> Prepared:
     """Offline steps with given (bfloat16) SVD factors: statistics, eq. 2,
-    migration (eq. 1), residual R = W_hat - L1 L2 and its 4-bit quantization."""
+    migration (eq. 1), residual R = W_hat - L1 L2 and its 4-bit quantization.
+    Rank 0 (L1 [K, 0], L2 [0, N]) is the smoothing-only case: R = W_hat."""
     W = np.asarray(W, dtype=np.float64)
     K, N = W.shape
     w_stat = weight_absmax(W)
-    s, inv_s = smoothing_factors(act_absmax, w_stat, alpha, s_min)
+    s, inv_s = smoothing_factors(act_absmax, w_stat, alpha, s_min, smooth)
     W_hat = migrate_weight(W, s)
     L1 = np.asarray(L1, dtype=np.float64)
     L2 = np.asarray(L2, dtype=np.float64)
@@ -172,14 +177,17 @@ def prepare_from_factors(W, bias, act_absmax, fmt: str, alpha: float, L1, L2, si
     return Prepared(fmt, K, N, L1.shape[1], alpha, s, inv_s, L1, L2, R, codes, scales, g_w, g_x, b, sigma)
 
 
-def prepare(W, bias, act_absmax, fmt: str, alpha: float, rank: int, s_min: float = float(S_MIN)) -> Prepared:
+def prepare(W, bias, act_absmax, fmt: str, alpha: float, rank: int, s_min: float = float(S_MIN),
+            smooth: bool = True) -> Prepared:
     """The three offline stages of section 2.1 in order: migrate (eq. 1, 2),
-    decompose (eq. 3, rank-r truncated SVD), quantize the residual."""
+    decompose (eq. 3, rank-r truncated SVD), quantize the residual.
+    rank = 0 skips the decomposition (smoothing only, the SmoothQuant special
+    case the entry's related terms name); smooth=False skips the migration."""
     W = np.asarray(W, dtype=np.float64)
-    s, _ = smoothing_factors(act_absmax, weight_absmax(W), alpha, s_min)
+    s, _ = smoothing_factors(act_absmax, weight_absmax(W), alpha, s_min, smooth)
     W_hat = migrate_weight(W, s)
     L1, L2, sigma = svd_factors(W_hat, rank)
-    return prepare_from_factors(W, bias, act_absmax, fmt, alpha, L1, L2, sigma, s_min)
+    return prepare_from_factors(W, bias, act_absmax, fmt, alpha, L1, L2, sigma, s_min, smooth)
 
 
 def smooth_activations(X, inv_s) -> np.ndarray:
@@ -236,10 +244,70 @@ def attach_lora(p: Prepared, A, B, scale: float) -> Prepared:
     The branch sees x_hat = X diag(s)^-1, so X A = x_hat (diag(s) A):
     L1' = [L1 | bf16(diag(s) A)], L2' = [L2 ; bf16(scale B)] (each product is
     exact in float64 and rounded once to bfloat16)."""
-    A = np.asarray(A, dtype=np.float64)
-    B = np.asarray(B, dtype=np.float64)
-    sA = bf16_round(p.s.astype(np.float64)[:, None] * A)
-    sB = bf16_round(np.float64(F32(scale)) * B)
+    sA, sB = lora_factors(p, A, B, scale)
     L1 = np.concatenate([p.L1, sA], axis=1)
     L2 = np.concatenate([p.L2, sB], axis=0)
     return dataclasses.replace(p, L1=L1, L2=L2, rank=L1.shape[1])
+
+
+def lora_factors(p: Prepared, A, B, scale: float):
+    """An adapter's branch factors: F = bf16(diag(s) A) [K, r_l] and
+    G = bf16(scale B) [r_l, N] (the branch sees x_hat = X diag(s)^-1)."""
+    A = np.asarray(A, dtype=np.float64)
+    B = np.asarray(B, dtype=np.float64)
+    F = bf16_round(p.s.astype(np.float64)[:, None] * A)
+    G = bf16_round(np.float64(F32(scale)) * B)
+    return F, G
+
+
+def forward_selected(p: Prepared, adapters: dict, X, row_mask) -> np.ndarray:
+    """Per-row adapter selection: row m of the output is the layer's output
+    plus, for every adapter slot a set in row_mask[m], that adapter's branch
+    product (x_hat F_a) G_a. `adapters` maps slot -> (F, G) from lora_factors;
+    p is the layer without adapters. All sums in float64."""
+    x_hat = smooth_activations(X, p.inv_s).astype(np.float64)
+    Y = forward(p, X).Y.copy()
+    mask = np.asarray(row_mask, dtype=np.int64)
+    for slot, (F, G) in adapters.items():
+        sel = ((mask >> slot) & 1).astype(bool)
+        if np.any(sel):
+            Y[sel] += (x_hat[sel] @ F) @ G
+    return Y
+
+
+# ---------------------------------------------------------------------------
+# the 4-bit weight-only baseline (W4A16) of the abstract's speed comparison
+# ---------------------------------------------------------------------------
+
+@dataclass
+class WeightOnly:
+    """W quantized alone (no smoothing, no branch): INT4 group 64 per output column."""
+
+    K: int
+    N: int
+    codes: np.ndarray  # int8 [N, K]
+    scales: np.ndarray  # float32 [N, K/64]
+    bias: np.ndarray  # float64 holding bf16 values [N]
+
+
+def prepare_weight_only(W, bias) -> WeightOnly:
+    """The weight-only baseline's offline step: the same symmetric INT4 group-64
+    quantizer as the W4A4 layer, applied to W itself, per output column."""
+    W = np.asarray(W, dtype=np.float64)
+    K, N = W.shape
+    codes, scales = quantize_int4_g64(np.ascontiguousarray(W.T).astype(F32))
+    b = np.zeros(N) if bias is None else np.asarray(bias, dtype=np.float64)
+    return WeightOnly(K, N, codes, scales, b)
+
+
+def dequantize_weight_only(p: WeightOnly) -> np.ndarray:
+    """w[n, k] = bf16(fp32(q[n, k] * scale[n, k / 64])): the bf16 operand the
+    activations meet (one float32 rounding of the product, then bf16)."""
+    q = p.codes.astype(F32).reshape(p.N, p.K // 64, 64)
+    prod = (q * p.scales.astype(F32)[:, :, None]).astype(F32)
+    return bf16_round(prod.reshape(p.N, p.K).astype(np.float64))
+
+
+def forward_weight_only(p: WeightOnly, X) -> np.ndarray:
+    """Y = X w^T + b in float64 with X in bf16 (the activations stay 16-bit)."""
+    return np.asarray(X, dtype=np.float64) @ dequantize_weight_only(p).T + p.bias[None, :]

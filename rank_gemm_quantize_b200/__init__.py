@@ -42,15 +42,20 @@ class SvdqError(RuntimeError):
         self.status = Status(status)
 
 
+NO_SMOOTHING = 1  # svdq_config.flags: s = 1 for every channel
+MAX_ADAPTERS = 8
+
+
 class _Config(ctypes.Structure):
     _fields_ = [("K", ctypes.c_int), ("N", ctypes.c_int), ("rank", ctypes.c_int), ("alpha", ctypes.c_float),
-                ("s_min", ctypes.c_float), ("fmt", ctypes.c_int)]
+                ("s_min", ctypes.c_float), ("fmt", ctypes.c_int), ("flags", ctypes.c_uint)]
 
 
 class _Info(ctypes.Structure):
     _fields_ = [("K", ctypes.c_int), ("N", ctypes.c_int), ("rank", ctypes.c_int), ("rank_pad", ctypes.c_int),
                 ("fmt", ctypes.c_int), ("alpha", ctypes.c_float), ("g_x", ctypes.c_float), ("g_w", ctypes.c_float),
-                ("t_scale", ctypes.c_float)]
+                ("t_scale", ctypes.c_float), ("base_rank", ctypes.c_int), ("flags", ctypes.c_uint),
+                ("adapter_slots", ctypes.c_uint), ("adapter_col_start", ctypes.c_int * (MAX_ADAPTERS + 1))]
 
 
 class _BlobHeader(ctypes.Structure):
@@ -72,7 +77,9 @@ SIGNATURES = {
     "svdq_linear_forward": [_VP, _VP, _I, _VP, _VP, _SZ, _VP],
     "svdq_linear_forward_profiled": [_VP, _VP, _I, _VP, _VP, _SZ, _VP, ctypes.POINTER(_VP)],
     "svdq_linear_forward_noalloc": [_VP, _VP, _I, _VP, _VP],
-    "svdq_attach_lora": [_VP, _VP, _VP, _I, _F, _VP],
+    "svdq_linear_forward_masked": [_VP, _VP, _I, _VP, _VP, _SZ, _VP, _VP],
+    "svdq_attach_lora": [_VP, _VP, _VP, _I, _F, _VP, ctypes.POINTER(_I)],
+    "svdq_detach_lora": [_VP, _I, _VP],
     "svdq_quantize_activations": [_VP, _VP, _I, _VP, _VP, _VP, _VP],
     "svdq_export_weights": [_VP, _VP, ctypes.POINTER(_SZ), _VP],
     "svdq_layer_get_info": [_VP, ctypes.POINTER(_Info)],
@@ -80,6 +87,11 @@ SIGNATURES = {
     "svdq_destroy": [_VP],
     "svdq_last_error": [],
     "svdq_selftest_bounded_wait": [ctypes.c_ulonglong, _VP],
+    "svdq_debug_fail_allocation": [ctypes.c_longlong],
+    "svdq_w4a16_prepare": [_VP, _VP, _I, _I, _VP, ctypes.POINTER(_VP)],
+    "svdq_w4a16_forward": [_VP, _VP, _I, _VP, _VP],
+    "svdq_w4a16_export": [_VP, _VP, _VP, _VP],
+    "svdq_w4a16_destroy": [_VP],
 }
 
 
@@ -91,7 +103,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     for name, args in SIGNATURES.items():
         fn = getattr(lib, name)
         fn.argtypes = args
-        fn.restype = ctypes.c_char_p if name == "svdq_last_error" else ctypes.c_int
+        fn.restype = {"svdq_last_error": ctypes.c_char_p, "svdq_debug_fail_allocation": None}.get(name, ctypes.c_int)
     return lib
 
 
@@ -149,20 +161,28 @@ class LayerInfo:
     g_x: float
     g_w: float
     t_scale: float
+    base_rank: int = 0
+    flags: int = 0
+    adapter_slots: int = 0
+    adapter_col_start: tuple = ()
 
 
 class Layer:
     """A prepared SVDQuant linear layer (owns its device buffers)."""
 
-    def __init__(self, handle: int):
+    def __init__(self, handle: int, device: Optional[torch.device] = None):
         self._h = ctypes.c_void_p(handle)
         self._ws: Optional[torch.Tensor] = None
+        self._info: Optional[LayerInfo] = None
+        self.device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
 
     @classmethod
     def prepare(cls, W: torch.Tensor, bias: Optional[torch.Tensor], act_absmax: torch.Tensor, fmt: str, rank: int,
-                alpha: float = 0.5, s_min: float = 1e-5, factors=None, stream=None) -> "Layer":
+                alpha: float = 0.5, s_min: float = 1e-5, factors=None, smooth: bool = True, stream=None) -> "Layer":
+        """Offline preparation; rank 0 gives the smoothing-only layer, smooth=False
+        keeps s = 1 (both ablations of the method)."""
         K, N = W.shape
-        cfg = _Config(K, N, rank, alpha, s_min, _FMT[fmt])
+        cfg = _Config(K, N, rank, alpha, s_min, _FMT[fmt], 0 if smooth else NO_SMOOTHING)
         out = ctypes.c_void_p()
         if factors is None:
             st = lib().svdq_prepare_weights(ctypes.byref(cfg), _ptr(W), _ptr(bias), _ptr(act_absmax), _stream(stream),
@@ -172,17 +192,42 @@ class Layer:
             st = lib().svdq_prepare_weights_with_factors(ctypes.byref(cfg), _ptr(W), _ptr(bias), _ptr(act_absmax),
                                                          _ptr(L1), _ptr(L2), _stream(stream), ctypes.byref(out))
         _check(st)
-        return cls(out.value)
+        return cls(out.value, W.device)
 
     def info(self) -> LayerInfo:
-        i = _Info()
-        _check(lib().svdq_layer_get_info(self._h, ctypes.byref(i)))
-        return LayerInfo(i.K, i.N, i.rank, i.rank_pad, _FMT_NAME[i.fmt], i.alpha, i.g_x, i.g_w, i.t_scale)
+        if self._info is None:
+            i = _Info()
+            _check(lib().svdq_layer_get_info(self._h, ctypes.byref(i)))
+            self._info = LayerInfo(i.K, i.N, i.rank, i.rank_pad, _FMT_NAME[i.fmt], i.alpha, i.g_x, i.g_w, i.t_scale,
+                                   i.base_rank, i.flags, i.adapter_slots, tuple(i.adapter_col_start))
+        return self._info
 
     def workspace_size(self, M: int) -> int:
         n = ctypes.c_size_t()
         _check(lib().svdq_workspace_size(self._h, M, ctypes.byref(n)))
         return n.value
+
+    def _check_io(self, X: torch.Tensor, out: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None) -> int:
+        """The shapes, dtypes and placement the C ABI assumes; the library reads
+        X through a tensor map built from the layer's K, so a narrower or
+        strided X would be read past its end."""
+        info = self.info()
+        if X.dim() != 2 or X.shape[1] != info.K:
+            raise ValueError(f"X must be [M, {info.K}], got {tuple(X.shape)}")
+        if X.dtype != torch.bfloat16 or not X.is_contiguous():
+            raise ValueError("X must be a contiguous bfloat16 tensor")
+        if X.device != self.device:
+            raise ValueError(f"X is on {X.device}, the layer on {self.device}")
+        if out is not None:
+            if tuple(out.shape) != (X.shape[0], info.N) or out.dtype != torch.bfloat16 or not out.is_contiguous():
+                raise ValueError(f"out must be a contiguous bfloat16 [{X.shape[0]}, {info.N}] tensor")
+            if out.device != self.device:
+                raise ValueError(f"out is on {out.device}, the layer on {self.device}")
+        if workspace is not None:
+            if workspace.dtype != torch.uint8 or not workspace.is_contiguous() or workspace.device != self.device:
+                raise ValueError("workspace must be a contiguous uint8 tensor on the layer's device")
+        return info.N
 
     def workspace(self, M: int, device=None) -> torch.Tensor:
         need = self.workspace_size(M)
@@ -192,8 +237,8 @@ class Layer:
 
     def forward(self, X: torch.Tensor, out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                 stream=None) -> torch.Tensor:
-        M, K = X.shape
-        N = self.info().N if out is None else out.shape[1]
+        N = self._check_io(X, out, workspace)
+        M = X.shape[0]
         if out is None:
             out = torch.empty(M, N, dtype=torch.bfloat16, device=X.device)
         ws = workspace if workspace is not None else self.workspace(M, X.device)
@@ -204,14 +249,16 @@ class Layer:
 
     def forward_noalloc(self, X: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
         """forward() on the library's fixed scratch array (no workspace, no allocation by the library)."""
+        N = self._check_io(X, out)
         M = X.shape[0]
         if out is None:
-            out = torch.empty(M, self.info().N, dtype=torch.bfloat16, device=X.device)
+            out = torch.empty(M, N, dtype=torch.bfloat16, device=X.device)
         _check(lib().svdq_linear_forward_noalloc(self._h, _ptr(X), M, _ptr(out), _stream(stream)))
         return out
 
     def forward_profiled(self, X: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor, events, stream=None):
         """forward() recording three torch.cuda.Event objects around its two kernels."""
+        self._check_io(X, out, workspace)
         arr = (ctypes.c_void_p * 3)(*[e.cuda_event for e in events])
         _check(lib().svdq_linear_forward_profiled(self._h, _ptr(X), X.shape[0], _ptr(out), _ptr(workspace),
                                                   workspace.numel(), _stream(stream), arr))
@@ -230,12 +277,38 @@ class Layer:
             codes = torch.empty(M_pad, K // 2, dtype=torch.uint8, device=dev)
             scales = torch.empty(M_pad // 128 * (K // 64) * 512, dtype=torch.uint8, device=dev)
         T = torch.empty(M_pad, info.rank_pad, dtype=torch.bfloat16, device=dev)
-        _check(lib().svdq_quantize_activations(self._h, _ptr(X), M, _ptr(codes), _ptr(scales), _ptr(T),
-                                               _stream(stream)))
+        _check(lib().svdq_quantize_activations(self._h, _ptr(X), M, _ptr(codes), _ptr(scales),
+                                               _ptr(T) if info.rank_pad else None, _stream(stream)))
         return codes, scales, T
 
-    def attach_lora(self, A: torch.Tensor, B: torch.Tensor, scale: float = 1.0, stream=None) -> None:
-        _check(lib().svdq_attach_lora(self._h, _ptr(A), _ptr(B), A.shape[1], scale, _stream(stream)))
+    def attach_lora(self, A: torch.Tensor, B: torch.Tensor, scale: float = 1.0, stream=None) -> int:
+        """Adds scale * X A B to the branch; returns the adapter's slot."""
+        self._info = None
+        slot = ctypes.c_int(-1)
+        _check(lib().svdq_attach_lora(self._h, _ptr(A), _ptr(B), A.shape[1], scale, _stream(stream),
+                                      ctypes.byref(slot)))
+        return slot.value
+
+    def detach_lora(self, slot: int, stream=None) -> None:
+        """Removes the adapter in `slot` (the branch returns to what it was without it)."""
+        self._info = None
+        _check(lib().svdq_detach_lora(self._h, slot, _stream(stream)))
+
+    def forward_masked(self, X: torch.Tensor, row_adapter_mask: torch.Tensor, out: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """forward() where row m uses the adapters whose slot bits are set in
+        row_adapter_mask[m] (int32/uint32 [M] on the layer's device)."""
+        N = self._check_io(X, out, workspace)
+        M = X.shape[0]
+        if (row_adapter_mask.dim() != 1 or row_adapter_mask.shape[0] != M or row_adapter_mask.element_size() != 4
+                or row_adapter_mask.device != self.device or not row_adapter_mask.is_contiguous()):
+            raise ValueError("row_adapter_mask must be a contiguous 32-bit [M] tensor on the layer's device")
+        if out is None:
+            out = torch.empty(M, N, dtype=torch.bfloat16, device=X.device)
+        ws = workspace if workspace is not None else self.workspace(M, X.device)
+        _check(lib().svdq_linear_forward_masked(self._h, _ptr(X), M, _ptr(out), _ptr(ws), ws.numel(),
+                                                _ptr(row_adapter_mask), _stream(stream)))
+        return out
 
     def export(self, stream=None) -> dict:
         """Canonical prepared weights (numpy arrays)."""
@@ -274,6 +347,52 @@ class Layer:
             lib().svdq_destroy(self._h)
         self._h = None
         self._ws = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class WeightOnlyLayer:
+    """The 4-bit weight-only (W4A16) baseline: INT4 group-64 weights, bf16
+    activations, dequantized on chip (include/svdq.h, svdq_w4a16_*)."""
+
+    def __init__(self, W: torch.Tensor, bias: Optional[torch.Tensor] = None, stream=None):
+        if W.dim() != 2 or W.dtype != torch.bfloat16 or not W.is_cuda or not W.is_contiguous():
+            raise ValueError("W must be a contiguous bfloat16 CUDA tensor [K, N]")
+        self.K, self.N = W.shape
+        self.device = W.device
+        out = ctypes.c_void_p()
+        _check(lib().svdq_w4a16_prepare(_ptr(W), _ptr(bias), self.K, self.N, _stream(stream), ctypes.byref(out)))
+        self._h = out
+
+    def forward(self, X: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        if X.dim() != 2 or X.shape[1] != self.K or X.dtype != torch.bfloat16 or not X.is_contiguous() \
+                or X.device != self.device:
+            raise ValueError(f"X must be a contiguous bfloat16 [M, {self.K}] tensor on {self.device}")
+        M = X.shape[0]
+        if out is None:
+            out = torch.empty(M, self.N, dtype=torch.bfloat16, device=X.device)
+        elif tuple(out.shape) != (M, self.N) or out.dtype != torch.bfloat16 or not out.is_contiguous():
+            raise ValueError(f"out must be a contiguous bfloat16 [{M}, {self.N}] tensor")
+        _check(lib().svdq_w4a16_forward(self._h, _ptr(X), M, _ptr(out), _stream(stream)))
+        return out
+
+    __call__ = forward
+
+    def export(self, stream=None):
+        """(codes uint8 [N, K/2] packed nibbles, scales float32 [K/64, N])."""
+        codes = np.zeros((self.N, self.K // 2), dtype=np.uint8)
+        scales = np.zeros((self.K // 64, self.N), dtype=np.float32)
+        _check(lib().svdq_w4a16_export(self._h, codes.ctypes.data, scales.ctypes.data, _stream(stream)))
+        return codes, scales
+
+    def close(self) -> None:
+        if self._h is not None and self._h.value:
+            lib().svdq_w4a16_destroy(self._h)
+        self._h = None
 
     def __del__(self):
         try:

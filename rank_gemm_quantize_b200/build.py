@@ -20,7 +20,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OUT = os.path.join(HERE, "libsvdq.so")
-SOURCES = ["svdq_api.cu", "act_quant.cu", "gemm_nvfp4.cu", "gemm_int4.cu", "prepare_kernels.cu", "noalloc.cu"]
+SOURCES = ["svdq_api.cu", "act_quant.cu", "gemm_nvfp4.cu", "gemm_int4.cu", "prepare_kernels.cu", "noalloc.cu",
+           "w4a16.cu"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr",

@@ -9,28 +9,38 @@
 // This kernel reads every X element from HBM once and produces all three in
 // the same pass.
 //
+// The branch input is computed as T = X (diag(s)^-1 L1): the layer keeps the
+// factor L1s = fp32(inv_s[k] L1[k, j]) as a bf16 pair hi + lo (hi = bf16(L1s),
+// lo = bf16(L1s - hi), about 16 significant bits together), so the tensor core
+// reads the bf16 X tile exactly as TMA brought it in and
+// T = X L1s_hi + X L1s_lo, an associative regrouping of X diag(s)^-1 L1.
+// The quantizers never have to build an MMA operand.
+//
 // Work split: CTA (b, s) owns rows [128 b, 128 b + 128) and the s-th of S
 // equal shares of K, walked in 64-column chunks. S is chosen so that the grid
 // fills the GPU in one wave; the CTAs never wait on one another. Per chunk:
-//   * warp 17 (one thread) streams the X tile [128 x 64], the L1^T slice
-//     [RP x 64] and the inv_s slice into a shared-memory ring with TMA / bulk
-//     copies (128-byte swizzle). The ring is as deep as shared memory allows
-//     (7 stages at RP = 32): X comes from HBM, and the loads in flight are
-//     what sets its bandwidth;
-//   * warps 0-15: each thread owns 16 consecutive elements of one row (a
-//     whole NVFP4 group; a quarter of an INT4 group, whose amax takes two
-//     shuffles). It smooths, quantizes, stores codes and scales, and writes
-//     x_hat as a bf16 high part and a bf16 remainder straight into a tcgen05
-//     K-major operand buffer;
-//   * one thread of warp 16 then issues tcgen05 kind::f16 MMAs
-//     (M = 128, N = RP, bf16 x bf16 -> fp32) of hi and lo against L1 into a
-//     TMEM accumulator, so x_hat enters the product with float accuracy.
+//   * warp 17 (one thread) streams the X tile [128 x 64], the two L1s^T
+//     slices [RP x 64] and the inv_s slice into a shared-memory ring with TMA
+//     and bulk copies (128-byte swizzle). The ring is as deep as shared memory
+//     allows (8 stages at RP = 32): X comes from HBM, and the bytes in flight
+//     set its bandwidth;
+//   * one thread of warp 16 issues the tcgen05 kind::f16 MMAs
+//     (M = 128, N = RP, bf16 x bf16 -> fp32) of the X tile against hi and lo
+//     into a TMEM accumulator;
+//   * warps 0-15: each thread owns 16 consecutive elements of one row, two
+//     chunks at a time for independent work (a whole NVFP4 group; a quarter
+//     of an INT4 group, whose amax takes two shuffles). It smooths,
+//     quantizes and stores codes and scales.
+// A stage is free again once the MMAs that read it have completed and all 16
+// quantizing warps have read it.
 // At the end each CTA parks its float partial product over its share of K in
 // the workspace and counts itself in on its row block's arrival counter; the
 // last of the S CTAs to arrive sums the S partials in share order (the same
 // sum whatever the arrival order), scales by t_scale, stores T as bf16 and
 // resets the counter for the next launch. With S = 1 the CTA stores T
-// directly.
+// directly. T columns that belong to a LoRA adapter a row has not selected
+// (per-row adapter mask) are stored as zero. RP = 0 (no branch: the
+// smoothing-only special case) compiles without TMEM, MMAs or T.
 //
 // Numerics of the quantizer match the CPU oracle operation by operation:
 // every product and quotient is a single IEEE round-to-nearest operation
@@ -55,22 +65,17 @@ constexpr int kMaxSplit = 16;      // K shares per row block (bounds the partial
 
 template <int RP>
 struct K1Shape {
-  static constexpr int kABufs = 2;                   // x_hat operand buffers
   static constexpr int kX = kRows * 128;             // X tile of a chunk (bf16, 64 cols)
-  static constexpr int kL = RP * 128;                // L1^T slice of a chunk
+  static constexpr int kL = RP * 128;                // one L1s^T slice (hi or lo) of a chunk
   static constexpr int kS = 256;                     // inv_s slice of a chunk
-  static constexpr int kStage = ((kX + kL + kS + 1023) / 1024) * 1024;  // 128-byte-swizzled TMA tiles start 1 KB-aligned
-  static constexpr int kAHalf = kRows * 128;         // one operand (hi or lo) of a chunk
-  static constexpr int kA = 2 * kAHalf;              // hi + lo MMA operand of a chunk
+  static constexpr int kStage = ((kX + 2 * kL + kS + 1023) / 1024) * 1024;  // swizzled TMA tiles start 1 KB-aligned
   static constexpr int kBudget = 232448 - 1024 - 512;  // dynamic shared memory, less alignment slack and barriers
-  static constexpr int kStagesFit = (kBudget - kABufs * kA) / kStage;
+  static constexpr int kStagesFit = kBudget / kStage;
   static constexpr int kStages = kStagesFit < 8 ? kStagesFit : 8;
-  static constexpr int kAOff = kStages * kStage;
-  static constexpr int kBarOff = kAOff + kABufs * kA;
+  static constexpr int kBarOff = kStages * kStage;
   static constexpr int kTotal = kBarOff + 256 + 1024;
   static_assert(kStages >= 2 && kTotal <= 232448, "shared memory budget");
   static_assert(kX % 1024 == 0 && kL % 1024 == 0, "TMA destinations stay 1024-byte aligned");
-  static constexpr int kMinBlocks = 1;
   static constexpr uint32_t kTmemCols = RP <= 32 ? 32 : (RP <= 64 ? 64 : (RP <= 128 ? 128 : 256));
 };
 
@@ -80,7 +85,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // Quantize this thread's 16 consecutive smoothed values v (row `row`, columns
 // k0 .. k0+15) and store their codes and group scale.
@@ -138,18 +142,60 @@ __device__ __forceinline__ void quantize16(const float (&v)[16], const ActQuantP
   }
 }
 
+// This thread's 16 smoothed values of one chunk: x_hat = fp32(x * inv_s),
+// one IEEE round-to-nearest product per element (packed pairs).
+__device__ __forceinline__ void smooth16(const uint8_t* xt, const float4* is4, uint32_t phys0, uint32_t phys1,
+                                         float (&v)[16]) {
+  const uint4 x0 = *reinterpret_cast<const uint4*>(xt + phys0);
+  const uint4 x1 = *reinterpret_cast<const uint4*>(xt + phys1);
+  const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float4 is = is4[e];
+    const float2 a = __fmul2_rn(make_float2(bf16_lo(w[2 * e]), bf16_hi(w[2 * e])), make_float2(is.x, is.y));
+    const float2 c = __fmul2_rn(make_float2(bf16_lo(w[2 * e + 1]), bf16_hi(w[2 * e + 1])), make_float2(is.z, is.w));
+    v[4 * e] = a.x;
+    v[4 * e + 1] = a.y;
+    v[4 * e + 2] = c.x;
+    v[4 * e + 3] = c.y;
+  }
+}
+
+// Whether branch column c of row `mask` is kept: the base factor's columns
+// always; an adapter's columns when the row selected its slot.
+__device__ __forceinline__ bool column_on(const ActQuantParams& p, uint32_t mask, int c) {
+  if (c < p.col_start[0]) return true;
+#pragma unroll
+  for (int s = 0; s < kMaxAdapters; ++s)
+    if (c < p.col_start[s + 1]) return (mask >> s) & 1u;
+  return true;  // padding columns (always zero)
+}
+
+// Stores 8 consecutive T columns c0 .. c0+7 of row r (scaled by t_scale, the
+// columns of unselected adapters zeroed).
+__device__ __forceinline__ void store_t8(const ActQuantParams& p, int RP, int r, int c0, const float (&a)[8]) {
+  float v[8];
+  // the mask has one entry per row of X; padding rows (r >= M) hold zeros anyway
+  const bool masked = p.row_mask != nullptr && r < p.M;
+  const uint32_t mask = masked ? __ldg(p.row_mask + r) : 0xFFFFFFFFu;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) v[e] = (masked && !column_on(p, mask, c0 + e)) ? 0.f : a[e] * p.t_scale;
+  const uint4 o = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                             pack_bf16x2(v[6], v[7]));
+  *reinterpret_cast<uint4*>(p.T + static_cast<size_t>(r) * RP + c0) = o;
+}
+
 template <int FMT, int RP>
-__global__ void __launch_bounds__(kThreads, K1Shape<RP>::kMinBlocks)
+__global__ void __launch_bounds__(kThreads, 1)
     act_quant_kernel(const ActQuantParams p, const __grid_constant__ ActQuantMaps maps) {
   using S = K1Shape<RP>;
+  constexpr bool kBranch = RP > 0;
   static_assert(RP % 32 == 0 && RP <= 256, "rank padding must be a multiple of 32, at most 256");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);  // [kStages] TMA landed
-  uint64_t* empty = full + S::kStages;                             // [kStages] MMA done with the stage
-  uint64_t* aready = empty + S::kStages;                           // [kABufs] operand written by warps 0-15
-  uint64_t* afree = aready + S::kABufs;                            // [kABufs] MMA done reading the operand
-  uint64_t* mma_done = afree + S::kABufs;
+  uint64_t* empty = full + S::kStages;                             // [kStages] MMAs and quantizers done with it
+  uint64_t* mma_done = empty + S::kStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* is_last = reinterpret_cast<volatile int*>(tmem_slot + 2);
@@ -168,39 +214,42 @@ __global__ void __launch_bounds__(kThreads, K1Shape<RP>::kMinBlocks)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S::kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int b = 0; b < S::kABufs; ++b) {
-      mbar_init(&aready[b], kQWarps);
-      mbar_init(&afree[b], 1);
+      mbar_init(&empty[s], kQWarps + (kBranch ? 1 : 0));
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == kMmaWarp) {
+  if (kBranch && warp == kMmaWarp) {
     tmem_alloc(tmem_slot, S::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = kBranch ? *tmem_slot : 0u;
 
   if (warp == kProdWarp) {
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tensormap(&maps.x);
-      prefetch_tensormap(&maps.l1t);
+      if (kBranch) {
+        prefetch_tensormap(&maps.l1h);
+        prefetch_tensormap(&maps.l1l);
+      }
       int j = 0;
       for (; j < nlocal; ++j) {
         const int s = j % S::kStages;
         if (!mbar_wait(&empty[s], ((j / S::kStages) & 1) ^ 1, abort_flag, p.status)) break;
         uint8_t* st = smem + s * S::kStage;
-        mbar_arrive_expect_tx(&full[s], S::kX + S::kL + kChunk * 4);
-        tma_load_2d(st, &maps.x, &full[s], (c_begin + j) * kChunk, m0);
-        tma_load_2d(st + S::kX, &maps.l1t, &full[s], (c_begin + j) * kChunk, 0);
-        bulk_load(st + S::kX + S::kL, p.inv_s + (c_begin + j) * kChunk, kChunk * 4, &full[s]);
+        const int kx = (c_begin + j) * kChunk;
+        mbar_arrive_expect_tx(&full[s], S::kX + 2 * S::kL + kChunk * 4);
+        tma_load_2d(st, &maps.x, &full[s], kx, m0);
+        if (kBranch) {
+          tma_load_2d(st + S::kX, &maps.l1h, &full[s], kx, 0);
+          tma_load_2d(st + S::kX + S::kL, &maps.l1l, &full[s], kx, 0);
+        }
+        bulk_load(st + S::kX + 2 * S::kL, p.inv_s + kx, kChunk * 4, &full[s]);
       }
       if (j < nlocal) {
         // gave up: let the copies still in flight land before the CTA exits
@@ -212,24 +261,22 @@ __global__ void __launch_bounds__(kThreads, K1Shape<RP>::kMinBlocks)
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_dense(kFmtF32, kFmtBF16, kFmtBF16, kRows, RP);
+    if (kBranch && lane == 0) {
+      const uint32_t idesc = idesc_dense(kFmtF32, kFmtBF16, kFmtBF16, kRows, RP > 0 ? RP : 32);
       for (int j = 0; j < nlocal; ++j) {
-        const int b = j % S::kABufs;
-        if (!mbar_wait(&aready[b], (j / S::kABufs) & 1, abort_flag, p.status)) break;
-        tc_fence_after();
         const int s = j % S::kStages;
-        const uint32_t a_hi = smem_u32(smem + S::kAOff + b * S::kA);
-        const uint32_t a_lo = a_hi + S::kAHalf;
-        const uint32_t bt = smem_u32(smem + s * S::kStage + S::kX);
+        if (!mbar_wait(&full[s], (j / S::kStages) & 1, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t xa = smem_u32(smem + s * S::kStage);
+        const uint32_t bh = xa + S::kX;
+        const uint32_t bl = bh + S::kL;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t bd = smem_desc(bt + 32 * ks, 16, 1024, kSw128);
-          mma_f16(tmem, smem_desc(a_hi + 32 * ks, 16, 1024, kSw128), bd, idesc, (j > 0 || ks > 0) ? 1u : 0u);
-          mma_f16(tmem, smem_desc(a_lo + 32 * ks, 16, 1024, kSw128), bd, idesc, 1u);
+          const uint64_t ad = smem_desc(xa + 32 * ks, 16, 1024, kSw128);
+          mma_f16(tmem, ad, smem_desc(bh + 32 * ks, 16, 1024, kSw128), idesc, (j > 0 || ks > 0) ? 1u : 0u);
+          mma_f16(tmem, ad, smem_desc(bl + 32 * ks, 16, 1024, kSw128), idesc, 1u);
         }
         tc_commit(&empty[s]);
-        tc_commit(&afree[b]);
       }
       tc_commit(mma_done);  // arrives once every MMA issued above has finished
     }
@@ -239,143 +286,129 @@ __global__ void __launch_bounds__(kThreads, K1Shape<RP>::kMinBlocks)
     const int seg = lane & 3;                 // 16-column segment of the chunk
     const int lrow = warp * 8 + (lane >> 2);  // row within the CTA
     const int row = m0 + lrow;
-    for (int j = 0; j < nlocal; ++j) {
-      const int s = j % S::kStages;
-      const int b = j % S::kABufs;
-      if (!mbar_wait(&full[s], (j / S::kStages) & 1, abort_flag, p.status)) break;
-      if (j >= S::kABufs && !mbar_wait(&afree[b], ((j / S::kABufs) & 1) ^ 1, abort_flag, p.status)) break;
-      const uint8_t* xt = smem + s * S::kStage;
-      const float4* is4 = reinterpret_cast<const float4*>(xt + S::kX + S::kL) + 4 * seg;
-      const uint32_t phys0 = lrow * 128 + (((2 * seg) ^ (lrow & 7)) * 16);
-      const uint32_t phys1 = lrow * 128 + (((2 * seg + 1) ^ (lrow & 7)) * 16);
-      const uint4 x0 = *reinterpret_cast<const uint4*>(xt + phys0);
-      const uint4 x1 = *reinterpret_cast<const uint4*>(xt + phys1);
-      const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-      float v[16];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float4 is = is4[e];
-        // one IEEE round-to-nearest product per element (packed pairs)
-        const float2 a = __fmul2_rn(make_float2(bf16_lo(w[2 * e]), bf16_hi(w[2 * e])), make_float2(is.x, is.y));
-        const float2 c = __fmul2_rn(make_float2(bf16_lo(w[2 * e + 1]), bf16_hi(w[2 * e + 1])), make_float2(is.z, is.w));
-        v[4 * e] = a.x;
-        v[4 * e + 1] = a.y;
-        v[4 * e + 2] = c.x;
-        v[4 * e + 3] = c.y;
-      }
-      quantize16<FMT>(v, p, row, (c_begin + j) * kChunk + 16 * seg, seg);
-      // x_hat = hi + lo with hi = bf16(x_hat) and lo = bf16(x_hat - hi) (the
-      // difference is exact in float), in the same 128-byte swizzle as the
-      // TMA tiles: the canonical tcgen05 K-major layout
-      uint32_t h[8], l[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        h[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-        const float2 d = __fadd2_rn(make_float2(v[2 * e], v[2 * e + 1]), make_float2(-bf16_lo(h[e]), -bf16_hi(h[e])));
-        l[e] = pack_bf16x2(d.x, d.y);
-      }
-      uint8_t* ad = smem + S::kAOff + b * S::kA;
-      *reinterpret_cast<uint4*>(ad + phys0) = make_uint4(h[0], h[1], h[2], h[3]);
-      *reinterpret_cast<uint4*>(ad + phys1) = make_uint4(h[4], h[5], h[6], h[7]);
-      *reinterpret_cast<uint4*>(ad + S::kAHalf + phys0) = make_uint4(l[0], l[1], l[2], l[3]);
-      *reinterpret_cast<uint4*>(ad + S::kAHalf + phys1) = make_uint4(l[4], l[5], l[6], l[7]);
-      fence_async_smem();  // make the generic-proxy writes visible to the tensor core
+    const uint32_t phys0 = lrow * 128 + (((2 * seg) ^ (lrow & 7)) * 16);
+    const uint32_t phys1 = lrow * 128 + (((2 * seg + 1) ^ (lrow & 7)) * 16);
+    constexpr int kIsOff = S::kX + 2 * S::kL;
+    int j = 0;
+    // two chunks per pass: two independent dependency chains per thread
+    for (; j + 1 < nlocal; j += 2) {
+      const int s0 = j % S::kStages, s1 = (j + 1) % S::kStages;
+      if (!mbar_wait(&full[s0], (j / S::kStages) & 1, abort_flag, p.status)) break;
+      if (!mbar_wait(&full[s1], ((j + 1) / S::kStages) & 1, abort_flag, p.status)) break;
+      const uint8_t* x0 = smem + s0 * S::kStage;
+      const uint8_t* x1 = smem + s1 * S::kStage;
+      float v0[16], v1[16];
+      smooth16(x0, reinterpret_cast<const float4*>(x0 + kIsOff) + 4 * seg, phys0, phys1, v0);
+      smooth16(x1, reinterpret_cast<const float4*>(x1 + kIsOff) + 4 * seg, phys0, phys1, v1);
       __syncwarp();
-      if (lane == 0) mbar_arrive(&aready[b]);
+      if (lane == 0) {
+        mbar_arrive(&empty[s0]);
+        mbar_arrive(&empty[s1]);
+      }
+      quantize16<FMT>(v0, p, row, (c_begin + j) * kChunk + 16 * seg, seg);
+      quantize16<FMT>(v1, p, row, (c_begin + j + 1) * kChunk + 16 * seg, seg);
+    }
+    if (j < nlocal) {
+      const int s0 = j % S::kStages;
+      if (mbar_wait(&full[s0], (j / S::kStages) & 1, abort_flag, p.status)) {
+        const uint8_t* x0 = smem + s0 * S::kStage;
+        float v0[16];
+        smooth16(x0, reinterpret_cast<const float4*>(x0 + kIsOff) + 4 * seg, phys0, phys1, v0);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s0]);
+        quantize16<FMT>(v0, p, row, (c_begin + j) * kChunk + 16 * seg, seg);
+      }
     }
   }
 
-  // ------------------------------------------------ this CTA's share of T
-  {
-    volatile int no_abort = 0;
-    mbar_wait(mma_done, 0, &no_abort, nullptr);
-  }
-  tc_fence_after();
-  const bool healthy = !*abort_flag;
-  // warp q may read TMEM lanes 32q .. 32q+31: rows 32q .. 32q+31 of the CTA
-  const int r = m0 + 32 * warp + lane;
-  const float sc = p.t_scale;
-  if (split == 1) {
-    if (warp < 4 && healthy) {
-#pragma unroll 1
-      for (int c0 = 0; c0 < RP; c0 += 32) {
-        uint32_t acc[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + c0, acc);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          const uint4 o = make_uint4(
-              pack_bf16x2(__uint_as_float(acc[e]) * sc, __uint_as_float(acc[e + 1]) * sc),
-              pack_bf16x2(__uint_as_float(acc[e + 2]) * sc, __uint_as_float(acc[e + 3]) * sc),
-              pack_bf16x2(__uint_as_float(acc[e + 4]) * sc, __uint_as_float(acc[e + 5]) * sc),
-              pack_bf16x2(__uint_as_float(acc[e + 6]) * sc, __uint_as_float(acc[e + 7]) * sc));
-          *reinterpret_cast<uint4*>(p.T + static_cast<size_t>(r) * RP + c0 + e) = o;
-        }
-      }
+  if (kBranch) {
+    // ---------------------------------------------- this CTA's share of T
+    {
+      volatile int no_abort = 0;
+      mbar_wait(mma_done, 0, &no_abort, nullptr);
     }
-  } else {
-    if (warp < 4) {
-      // park this share's partial; a CTA that gave up parks zeros, so the
-      // arrival count stays right and the status word reports the failure
-      float* dst = p.Tpart + (static_cast<size_t>(sh) * p.M_pad + r) * RP;
+    tc_fence_after();
+    const bool healthy = !*abort_flag;
+    // warp q may read TMEM lanes 32q .. 32q+31: rows 32q .. 32q+31 of the CTA
+    const int r = m0 + 32 * warp + lane;
+    if (split == 1) {
+      if (warp < 4 && healthy) {
 #pragma unroll 1
-      for (int c0 = 0; c0 < RP; c0 += 32) {
-        uint32_t acc[32];
-        if (healthy) {
+        for (int c0 = 0; c0 < RP; c0 += 32) {
+          uint32_t acc[32];
           tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + c0, acc);
           tmem_ld_wait();
-        } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) acc[e] = 0u;
+          for (int e = 0; e < 32; e += 8) {
+            float a[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) a[i] = __uint_as_float(acc[e + i]);
+            store_t8(p, RP, r, c0 + e, a);
+          }
         }
-#pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(dst + c0 + e) = make_float4(__uint_as_float(acc[e]), __uint_as_float(acc[e + 1]),
-                                                                 __uint_as_float(acc[e + 2]), __uint_as_float(acc[e + 3]));
       }
-      __threadfence();  // the partial is visible device-wide before this CTA counts itself in
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      const int prev = atomicAdd(p.counters + rb, 1);
-      const int last = prev == split - 1;
-      if (last) p.counters[rb] = 0;  // every share has arrived: ready for the next launch
-      *is_last = last;
-    }
-    __syncthreads();
-    if (*is_last && warp < kQWarps) {
-      __threadfence();  // acquire side: the other shares' partials are visible
-      // all quantizing threads sum: one 8-column slice of one row per item,
-      // four shares' loads in flight at a time, shares added in order
-      constexpr int kSlices = RP / 8;
+    } else {
+      if (warp < 4) {
+        // park this share's partial; a CTA that gave up parks zeros, so the
+        // arrival count stays right and the status word reports the failure
+        float* dst = p.Tpart + (static_cast<size_t>(sh) * p.M_pad + r) * RP;
 #pragma unroll 1
-      for (int item = threadIdx.x; item < kRows * kSlices; item += kQWarps * 32) {
-        const int rr = m0 + item / kSlices;
-        const int c0 = (item % kSlices) * 8;
-        const float* src = p.Tpart + static_cast<size_t>(rr) * RP + c0;
-        const size_t stride = static_cast<size_t>(p.M_pad) * RP;
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-        for (int t0 = 0; t0 < split; t0 += 4) {
-          float4 u[4], w[4];
+        for (int c0 = 0; c0 < RP; c0 += 32) {
+          uint32_t acc[32];
+          if (healthy) {
+            tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + c0, acc);
+            tmem_ld_wait();
+          } else {
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            if (t0 + t < split) {
-              u[t] = __ldcg(reinterpret_cast<const float4*>(src + (t0 + t) * stride));
-              w[t] = __ldcg(reinterpret_cast<const float4*>(src + (t0 + t) * stride + 4));
-            }
+            for (int e = 0; e < 32; ++e) acc[e] = 0u;
           }
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            if (t0 + t < split) {  // share order: the same sum whatever the arrival order
-              acc[0] += u[t].x; acc[1] += u[t].y; acc[2] += u[t].z; acc[3] += u[t].w;
-              acc[4] += w[t].x; acc[5] += w[t].y; acc[6] += w[t].z; acc[7] += w[t].w;
-            }
-          }
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + c0 + e) = make_float4(__uint_as_float(acc[e]), __uint_as_float(acc[e + 1]),
+                                                                   __uint_as_float(acc[e + 2]), __uint_as_float(acc[e + 3]));
         }
-        const uint4 o = make_uint4(pack_bf16x2(acc[0] * sc, acc[1] * sc), pack_bf16x2(acc[2] * sc, acc[3] * sc),
-                                   pack_bf16x2(acc[4] * sc, acc[5] * sc), pack_bf16x2(acc[6] * sc, acc[7] * sc));
-        *reinterpret_cast<uint4*>(p.T + static_cast<size_t>(rr) * RP + c0) = o;
+        __threadfence();  // the partial is visible device-wide before this CTA counts itself in
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        const int prev = atomicAdd(p.counters + rb, 1);
+        const int last = prev == split - 1;
+        if (last) p.counters[rb] = 0;  // every share has arrived: ready for the next launch
+        *is_last = last;
+      }
+      __syncthreads();
+      if (*is_last && warp < kQWarps) {
+        __threadfence();  // acquire side: the other shares' partials are visible
+        // all quantizing threads sum: one 8-column slice of one row per item,
+        // four shares' loads in flight at a time, shares added in order
+        constexpr int kSlices = RP / 8;
+#pragma unroll 1
+        for (int item = threadIdx.x; item < kRows * kSlices; item += kQWarps * 32) {
+          const int rr = m0 + item / kSlices;
+          const int c0 = (item % kSlices) * 8;
+          const float* src = p.Tpart + static_cast<size_t>(rr) * RP + c0;
+          const size_t stride = static_cast<size_t>(p.M_pad) * RP;
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+          for (int t0 = 0; t0 < split; t0 += 4) {
+            float4 u[4], w[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              if (t0 + t < split) {
+                u[t] = __ldcg(reinterpret_cast<const float4*>(src + (t0 + t) * stride));
+                w[t] = __ldcg(reinterpret_cast<const float4*>(src + (t0 + t) * stride + 4));
+              }
+            }
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              if (t0 + t < split) {  // share order: the same sum whatever the arrival order
+                acc[0] += u[t].x; acc[1] += u[t].y; acc[2] += u[t].z; acc[3] += u[t].w;
+                acc[4] += w[t].x; acc[5] += w[t].y; acc[6] += w[t].z; acc[7] += w[t].w;
+              }
+            }
+          }
+          store_t8(p, RP, rr, c0, acc);
+        }
       }
     }
   }
@@ -383,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, K1Shape<RP>::kMinBlocks)
   // ------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (kBranch && warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, S::kTmemCols);
   }
@@ -406,7 +439,10 @@ template <int FMT, int RP>
 int resident_ctas() {
   using S = K1Shape<RP>;
   auto kern = act_quant_kernel<FMT, RP>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal) != cudaSuccess) return 1;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal) != cudaSuccess) {
+    cudaGetLastError();
+    return 1;
+  }
   int n = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, S::kTotal) != cudaSuccess || n < 1) {
     cudaGetLastError();
@@ -415,17 +451,16 @@ int resident_ctas() {
   return n;
 }
 
+#define SVDQ_RP_CASES(F) F(0) F(32) F(64) F(96) F(128) F(160) F(192) F(224) F(256)
+
 template <int FMT>
 int resident_fmt(int rp) {
   switch (rp) {
-    case 32: return resident_ctas<FMT, 32>();
-    case 64: return resident_ctas<FMT, 64>();
-    case 96: return resident_ctas<FMT, 96>();
-    case 128: return resident_ctas<FMT, 128>();
-    case 160: return resident_ctas<FMT, 160>();
-    case 192: return resident_ctas<FMT, 192>();
-    case 224: return resident_ctas<FMT, 224>();
-    case 256: return resident_ctas<FMT, 256>();
+#define SVDQ_CASE(R) \
+  case R:            \
+    return resident_ctas<FMT, R>();
+    SVDQ_RP_CASES(SVDQ_CASE)
+#undef SVDQ_CASE
     default: return 1;
   }
 }
@@ -433,14 +468,11 @@ int resident_fmt(int rp) {
 template <int FMT>
 cudaError_t launch_fmt(const ActQuantParams& p, const ActQuantMaps& maps, int rp, cudaStream_t stream) {
   switch (rp) {
-    case 32: return launch_rp<FMT, 32>(p, maps, stream);
-    case 64: return launch_rp<FMT, 64>(p, maps, stream);
-    case 96: return launch_rp<FMT, 96>(p, maps, stream);
-    case 128: return launch_rp<FMT, 128>(p, maps, stream);
-    case 160: return launch_rp<FMT, 160>(p, maps, stream);
-    case 192: return launch_rp<FMT, 192>(p, maps, stream);
-    case 224: return launch_rp<FMT, 224>(p, maps, stream);
-    case 256: return launch_rp<FMT, 256>(p, maps, stream);
+#define SVDQ_CASE(R) \
+  case R:            \
+    return launch_rp<FMT, R>(p, maps, stream);
+    SVDQ_RP_CASES(SVDQ_CASE)
+#undef SVDQ_CASE
     default: return cudaErrorInvalidValue;
   }
 }
@@ -449,18 +481,15 @@ cudaError_t launch_fmt(const ActQuantParams& p, const ActQuantMaps& maps, int rp
 
 int act_quant_box_rows() { return kRows; }
 
-int act_quant_split(int M_pad, int K, int fmt, int rp, int sms) {
-  // CTAs that fit on the GPU at once, divided among the 64-row blocks; each
+int act_quant_resident(int fmt, int rp) {
+  return fmt == SVDQ_INT4_G64 ? resident_fmt<SVDQ_INT4_G64>(rp) : resident_fmt<SVDQ_NVFP4_G16>(rp);
+}
+
+int act_quant_split(int M_pad, int K, int per_sm, int sms) {
+  // CTAs that fit on the GPU at once, divided among the 128-row blocks; each
   // CTA keeps at least one chunk, and at most kMaxSplit partials are summed.
-  // resident CTAs per SM for (format, rank padding), queried once per process
-  static int cache[2][9] = {};
-  const int fi = fmt == SVDQ_INT4_G64 ? 0 : 1, ri = rp / 32;
-  if (ri < 1 || ri > 8) return 1;
-  if (cache[fi][ri] == 0)
-    cache[fi][ri] = fmt == SVDQ_INT4_G64 ? resident_fmt<SVDQ_INT4_G64>(rp) : resident_fmt<SVDQ_NVFP4_G16>(rp);
-  const int per_sm = cache[fi][ri];
   const int row_blocks = M_pad / kRows;
-  int split = (sms * per_sm) / row_blocks;
+  int split = (sms * (per_sm < 1 ? 1 : per_sm)) / row_blocks;
   const int nchunks = K / kChunk;
   if (split > nchunks) split = nchunks;
   if (split > kMaxSplit) split = kMaxSplit;
@@ -470,7 +499,7 @@ int act_quant_split(int M_pad, int K, int fmt, int rp, int sms) {
 cudaError_t launch_act_quant(const ActQuantParams& p, const ActQuantMaps& maps, int fmt, int rp,
                              cudaStream_t stream) {
   if (p.M_pad % 128 != 0 || p.K % 128 != 0 || p.split < 1 || p.M_pad / kRows > kMaxRowBlocks ||
-      (p.split > 1 && (!p.Tpart || !p.counters)))
+      (rp > 0 && p.split > 1 && (!p.Tpart || !p.counters)) || (rp > 0 && !p.T))
     return cudaErrorInvalidValue;
   if (fmt == SVDQ_INT4_G64) return launch_fmt<SVDQ_INT4_G64>(p, maps, rp, stream);
   return launch_fmt<SVDQ_NVFP4_G16>(p, maps, rp, stream);

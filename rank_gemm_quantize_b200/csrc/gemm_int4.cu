@@ -132,8 +132,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       prefetch_tensormap(&maps.a);
       prefetch_tensormap(&maps.b);
-      prefetch_tensormap(&maps.t);
-      prefetch_tensormap(&maps.l2);
+      if (n_lr > 0) {  // no branch (rank 0): its maps are never read
+        prefetch_tensormap(&maps.t);
+        prefetch_tensormap(&maps.l2);
+      }
       bool ok = true;
       int it = 0;  // k-tiles issued by this CTA over all its tiles
       int gs = 0;  // scale vectors issued by this CTA over all its tiles
@@ -258,7 +260,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       float2 acc[kCols / 2];
 #pragma unroll
       for (int j = 0; j < kCols / 2; ++j) acc[j] = make_float2(0.f, 0.f);
-      for (int g = 0; g <= n_groups && ok; ++g, ++ga) {
+      // the groups, then (with a branch) one pass for the low-rank product
+      const int n_acc = n_groups + (n_lr > 0 ? 1 : 0);
+      for (int g = 0; g < n_acc && ok; ++g, ++ga) {
         const bool branch = (g == n_groups);
         const int ws = gs % kSwSlots;
         if (!branch) {

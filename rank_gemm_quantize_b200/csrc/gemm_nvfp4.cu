@@ -129,8 +129,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       prefetch_tensormap(&maps.a);
       prefetch_tensormap(&maps.b);
-      prefetch_tensormap(&maps.t);
-      prefetch_tensormap(&maps.l2);
+      if (n_lr > 0) {  // no branch (rank 0): its maps are never read
+        prefetch_tensormap(&maps.t);
+        prefetch_tensormap(&maps.l2);
+      }
       bool ok = true;
       int it = 0;          // k-tiles issued over all tiles of this CTA
       int ti = 0;          // tiles of this CTA

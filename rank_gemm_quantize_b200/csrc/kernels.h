@@ -9,12 +9,20 @@
 
 namespace svdq {
 
+// A 2-D tiled TMA map over a row-major [outer, inner] tensor (row_bytes
+// between rows), box {box_inner, box_outer}; false if encoding failed.
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw);
+
+// LoRA adapter slots a layer can hold at once (bit s of a row's adapter mask
+// selects slot s).
+constexpr int kMaxAdapters = 8;
+
 // ---------------------------------------------------------------- K1
 struct ActQuantParams {
   const __nv_bfloat16* X;  // [M, K] row-major
   int M, K, M_pad;         // M_pad = roundup(M, 128)
   const float* inv_s;      // [K]
-  const __nv_bfloat16* L1T;  // [RP, K]: transposed, zero-padded down-projection factor
   uint8_t* codes;          // INT4: [M_pad, K] E4M3 bytes of the integer codes; NVFP4: [M_pad, K/2] packed E2M1
   void* scales;            // INT4: float [K/64][M_pad]; NVFP4: scale-factor atoms [M_pad/128][K/64][512]
   __nv_bfloat16* T;        // [M_pad, RP] bf16 = t_scale * (x_hat L1)
@@ -25,14 +33,24 @@ struct ActQuantParams {
   float denom;             // NVFP4: fp32(6 * g_x)
   float t_scale;           // 1 (INT4) or 1 / (g_x g_w) (NVFP4)
   int* status;             // device status word (kDevTimeout on a given-up wait)
+  // Per-row LoRA adapter selection: bit s of row_mask[m] keeps the T columns
+  // of adapter slot s for row m ([col_start[s], col_start[s+1])); the base
+  // factor's columns [0, col_start[0]) are always kept. NULL keeps everything.
+  const uint32_t* row_mask;  // [M] or NULL
+  int col_start[kMaxAdapters + 1];
 };
 struct ActQuantMaps {
-  CUtensorMap x;    // X [M, K] bf16, box {64, 32}, 128-byte swizzle
-  CUtensorMap l1t;  // L1T [RP, K] bf16, box {64, RP}, 128-byte swizzle
+  CUtensorMap x;    // X [M, K] bf16, box {64, 128}, 128-byte swizzle
+  CUtensorMap l1h;  // L1s^T high part [RP, K] bf16, box {64, RP}, 128-byte swizzle
+  CUtensorMap l1l;  // L1s^T low part  [RP, K] bf16, box {64, RP}, 128-byte swizzle
 };
 int act_quant_box_rows();
-// K shares per 128-row block for M_pad rows: the grid fills the GPU in one wave.
-int act_quant_split(int M_pad, int K, int fmt, int rp, int sms);
+// Resident activation-kernel CTAs per SM for (format, rank padding) on the
+// current device (an occupancy query; call it once per layer, not per launch).
+int act_quant_resident(int fmt, int rp);
+// K shares per 128-row block for M_pad rows, so that the grid fills the GPU in
+// one wave: a pure function of its arguments.
+int act_quant_split(int M_pad, int K, int per_sm, int sms);
 // Row blocks the per-layer arrival counters cover (M_pad / 128 at most this).
 constexpr int kMaxRowBlocks = 65536;
 cudaError_t launch_act_quant(const ActQuantParams& p, const ActQuantMaps& maps, int fmt, int rp, cudaStream_t stream);
@@ -80,12 +98,12 @@ cudaError_t launch_quant_weight_int4(const float* R, int K, int N, int N_pad, ui
                                      cudaStream_t st);
 cudaError_t launch_quant_weight_nvfp4(const float* R, int K, int N, int N_pad, const unsigned int* amax_bits,
                                       uint8_t* codes4, uint8_t* sf_atoms, float* g_w_out, cudaStream_t st);
-cudaError_t launch_build_branch(const __nv_bfloat16* L1, const __nv_bfloat16* L2, int K, int N, int rank, int RP,
-                                int N_pad, __nv_bfloat16* L1T, __nv_bfloat16* L2T, cudaStream_t st);
-cudaError_t launch_lora_concat(const __nv_bfloat16* L1T_old, const __nv_bfloat16* L2T_old, int K, int N, int N_pad,
-                               int rank_old, int RP_old, const float* s_k, const __nv_bfloat16* A,
-                               const __nv_bfloat16* B, int r_l, float scale, int RP_new, __nv_bfloat16* L1T,
-                               __nv_bfloat16* L2T, cudaStream_t st);
+// Writes one block of branch columns [c0, c0 + rb) (see prepare_kernels.cu).
+cudaError_t launch_assemble_block(const __nv_bfloat16* F, const __nv_bfloat16* G, int rb, int c0, int K, int N,
+                                  int RP, const float* inv_s, __nv_bfloat16* L1T, __nv_bfloat16* L1sTh,
+                                  __nv_bfloat16* L1sTl, __nv_bfloat16* L2T, cudaStream_t st);
+cudaError_t launch_lora_factors(const __nv_bfloat16* A, const __nv_bfloat16* B, int K, int N, int r_l, float scale,
+                                const float* s_k, __nv_bfloat16* F, __nv_bfloat16* G, cudaStream_t st);
 cudaError_t launch_wait_selftest(int* status, unsigned long long limit_ns, cudaStream_t st);
 
 }  // namespace svdq

@@ -28,9 +28,13 @@ void set_last_error(const std::string& msg);
 
 namespace {
 
-// Largest workspace the array holds: enough for M x K = 4608 x 3072 in either
-// format up to rank 128 (at rank 32: about 17 MiB for INT4, 10 MiB for
-// NVFP4, including the activation kernel's float partials of T).
+// Largest workspace the array holds. What a call needs is svdq_workspace_size:
+// the activation codes and scales, T, and the activation kernel's float
+// partials of T, whose count is the kernel's K split (SMs x resident CTAs per
+// SM / 128-row blocks, at most 16). With one resident CTA per SM that split is
+// 4 at 4608 rows on 148 SMs, and the 4608 x 3072 attention projection then
+// needs about 25 MiB (INT4) or 18 MiB (NVFP4) at rank 128, 17 / 10 MiB at
+// rank 32. Anything larger is refused below, whatever the shape.
 constexpr size_t kScratchBytes = size_t(32) << 20;
 
 constexpr int kMaxDevices = 64;

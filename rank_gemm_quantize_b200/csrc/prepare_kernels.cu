@@ -213,56 +213,52 @@ __global__ void quant_w_nvfp4_kernel(const float* R, int K, int N, const unsigne
   sf_atoms[atom * 512 + (n & 31) * 16 + ((n >> 5) & 3) * 4 + (b & 3)] = static_cast<uint8_t>(sb);
 }
 
-// L1 [K, rank] -> L1T [RP, K]; L2 [rank, N] -> L2T [N_pad, RP]; zero padding.
-__global__ void build_branch_kernel(const __nv_bfloat16* L1, const __nv_bfloat16* L2, int K, int N, int rank, int RP,
-                                    int N_pad, __nv_bfloat16* L1T, __nv_bfloat16* L2T) {
+// One block of the low-rank branch (the base factors, or one LoRA adapter)
+// written at branch columns [c0, c0 + rb):
+//   L1T [RP, K]   <- F^T         (the canonical input-side factor)
+//   L1sTh, L1sTl  <- hi / lo of fp32(inv_s[k] * F[k, j]): hi = bf16(v),
+//                    lo = bf16(v - hi) (the difference is exact in float), the
+//                    factor with 1/s folded in that the activation kernel uses
+//   L2T [N_pad, RP] <- G^T       (the output-side factor)
+// F is [K, rb] and G is [rb, N], both row-major bf16. Columns outside every
+// block stay as the caller zeroed them.
+__global__ void assemble_block_kernel(const __nv_bfloat16* F, const __nv_bfloat16* G, int rb, int c0, int K, int N,
+                                      int RP, const float* inv_s, __nv_bfloat16* L1T, __nv_bfloat16* L1sTh,
+                                      __nv_bfloat16* L1sTl, __nv_bfloat16* L2T) {
   const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const size_t n1 = static_cast<size_t>(RP) * K;
-  const size_t n2 = static_cast<size_t>(N_pad) * RP;
+  const size_t n1 = static_cast<size_t>(rb) * K;
+  const size_t n2 = static_cast<size_t>(rb) * N;
   if (i < n1) {
     const int j = static_cast<int>(i / K), k = static_cast<int>(i % K);
-    L1T[i] = j < rank ? L1[static_cast<size_t>(k) * rank + j] : __ushort_as_bfloat16(0);
+    const __nv_bfloat16 f = F[static_cast<size_t>(k) * rb + j];
+    const size_t o = static_cast<size_t>(c0 + j) * K + k;
+    L1T[o] = f;
+    const float v = __fmul_rn(inv_s[k], __bfloat162float(f));
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    L1sTh[o] = hi;
+    L1sTl[o] = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(hi)));
   } else if (i < n1 + n2) {
     const size_t t = i - n1;
-    const int n = static_cast<int>(t / RP), j = static_cast<int>(t % RP);
-    L2T[t] = (j < rank && n < N) ? L2[static_cast<size_t>(j) * N + n] : __ushort_as_bfloat16(0);
+    const int j = static_cast<int>(t / N), n = static_cast<int>(t % N);
+    L2T[static_cast<size_t>(n) * RP + c0 + j] = G[t];
   }
 }
 
-// Concatenate a LoRA (A [K, r_l], B [r_l, N], scale) into the branch:
-// L1' = [L1 | bf16(diag(s) A)], L2' = [L2 ; bf16(scale B)]; each product is
-// exact in float64 and rounded once.
-__global__ void lora_concat_kernel(const __nv_bfloat16* L1T_old, const __nv_bfloat16* L2T_old, int K, int N, int N_pad,
-                                   int rank_old, int RP_old, const float* s, const __nv_bfloat16* A,
-                                   const __nv_bfloat16* B, int r_l, float scale, int RP_new, __nv_bfloat16* L1T,
-                                   __nv_bfloat16* L2T) {
+// The factors of a LoRA adapter as the branch sees them. The branch input is
+// x_hat = X diag(s)^-1, so X A = x_hat (diag(s) A): F = bf16(s[k] * A[k, j])
+// [K, r_l] and G = bf16(scale * B[j, n]) [r_l, N]; each product is exact in
+// float64 and rounded once.
+__global__ void lora_factors_kernel(const __nv_bfloat16* A, const __nv_bfloat16* B, int K, int N, int r_l, float scale,
+                                    const float* s, __nv_bfloat16* F, __nv_bfloat16* G) {
   const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const size_t n1 = static_cast<size_t>(RP_new) * K;
-  const size_t n2 = static_cast<size_t>(N_pad) * RP_new;
-  const __nv_bfloat16 zero = __ushort_as_bfloat16(0);
+  const size_t n1 = static_cast<size_t>(K) * r_l;
+  const size_t n2 = static_cast<size_t>(r_l) * N;
   if (i < n1) {
-    const int j = static_cast<int>(i / K), k = static_cast<int>(i % K);
-    __nv_bfloat16 v = zero;
-    if (j < rank_old) {
-      v = L1T_old[static_cast<size_t>(j) * K + k];
-    } else if (j < rank_old + r_l) {
-      const double a = static_cast<double>(__bfloat162float(A[static_cast<size_t>(k) * r_l + (j - rank_old)]));
-      v = bf16_from_double(static_cast<double>(s[k]) * a);
-    }
-    L1T[i] = v;
+    const int k = static_cast<int>(i / r_l);
+    F[i] = bf16_from_double(static_cast<double>(s[k]) * static_cast<double>(__bfloat162float(A[i])));
   } else if (i < n1 + n2) {
     const size_t t = i - n1;
-    const int n = static_cast<int>(t / RP_new), j = static_cast<int>(t % RP_new);
-    __nv_bfloat16 v = zero;
-    if (n < N) {
-      if (j < rank_old) {
-        v = L2T_old[static_cast<size_t>(n) * RP_old + j];
-      } else if (j < rank_old + r_l) {
-        const double b = static_cast<double>(__bfloat162float(B[static_cast<size_t>(j - rank_old) * N + n]));
-        v = bf16_from_double(static_cast<double>(scale) * b);
-      }
-    }
-    L2T[t] = v;
+    G[t] = bf16_from_double(static_cast<double>(scale) * static_cast<double>(__bfloat162float(B[t])));
   }
 }
 
@@ -340,19 +336,18 @@ cudaError_t launch_quant_weight_nvfp4(const float* R, int K, int N, int N_pad, c
   quant_w_nvfp4_kernel<<<grid, 128, 0, st>>>(R, K, N, amax_bits, codes4, sf_atoms, g_w_out);
   return cudaGetLastError();
 }
-cudaError_t launch_build_branch(const __nv_bfloat16* L1, const __nv_bfloat16* L2, int K, int N, int rank, int RP,
-                                int N_pad, __nv_bfloat16* L1T, __nv_bfloat16* L2T, cudaStream_t st) {
-  const size_t n = static_cast<size_t>(RP) * K + static_cast<size_t>(N_pad) * RP;
-  build_branch_kernel<<<blocks_for(n, 256), 256, 0, st>>>(L1, L2, K, N, rank, RP, N_pad, L1T, L2T);
+cudaError_t launch_assemble_block(const __nv_bfloat16* F, const __nv_bfloat16* G, int rb, int c0, int K, int N,
+                                  int RP, const float* inv_s, __nv_bfloat16* L1T, __nv_bfloat16* L1sTh,
+                                  __nv_bfloat16* L1sTl, __nv_bfloat16* L2T, cudaStream_t st) {
+  const size_t n = static_cast<size_t>(rb) * (K + N);
+  if (n == 0) return cudaSuccess;
+  assemble_block_kernel<<<blocks_for(n, 256), 256, 0, st>>>(F, G, rb, c0, K, N, RP, inv_s, L1T, L1sTh, L1sTl, L2T);
   return cudaGetLastError();
 }
-cudaError_t launch_lora_concat(const __nv_bfloat16* L1T_old, const __nv_bfloat16* L2T_old, int K, int N, int N_pad,
-                               int rank_old, int RP_old, const float* s_k, const __nv_bfloat16* A,
-                               const __nv_bfloat16* B, int r_l, float scale, int RP_new, __nv_bfloat16* L1T,
-                               __nv_bfloat16* L2T, cudaStream_t st) {
-  const size_t n = static_cast<size_t>(RP_new) * K + static_cast<size_t>(N_pad) * RP_new;
-  lora_concat_kernel<<<blocks_for(n, 256), 256, 0, st>>>(L1T_old, L2T_old, K, N, N_pad, rank_old, RP_old, s_k, A, B,
-                                                         r_l, scale, RP_new, L1T, L2T);
+cudaError_t launch_lora_factors(const __nv_bfloat16* A, const __nv_bfloat16* B, int K, int N, int r_l, float scale,
+                                const float* s_k, __nv_bfloat16* F, __nv_bfloat16* G, cudaStream_t st) {
+  const size_t n = static_cast<size_t>(r_l) * (K + N);
+  lora_factors_kernel<<<blocks_for(n, 256), 256, 0, st>>>(A, B, K, N, r_l, scale, s_k, F, G);
   return cudaGetLastError();
 }
 cudaError_t launch_wait_selftest(int* status, unsigned long long limit_ns, cudaStream_t st) {

@@ -29,19 +29,6 @@ svdq_status fail(svdq_status st, const std::string& msg) {
 namespace svdq {
 // Lets other translation units of the library report through svdq_last_error.
 void set_last_error(const std::string& msg) { g_last_error = msg; }
-}  // namespace svdq
-
-namespace {
-
-#define CUDA_TRY(expr)                                                                              \
-  do {                                                                                              \
-    cudaError_t e__ = (expr);                                                                       \
-    if (e__ != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string(#expr) + ": " + cudaGetErrorString(e__)); \
-  } while (0)
-
-inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
-inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
-inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -69,6 +56,20 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+}  // namespace svdq
+
+namespace {
+
+#define CUDA_TRY(expr)                                                                              \
+  do {                                                                                              \
+    cudaError_t e__ = (expr);                                                                       \
+    if (e__ != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string(#expr) + ": " + cudaGetErrorString(e__)); \
+  } while (0)
+
+inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 // Weight-side padding: every GEMM tile width divides it, so per-tile scale
 // copies never leave the buffers.
@@ -114,20 +115,36 @@ struct WsLayout {
 struct svdq_layer {
   int device = 0;
   int sms = 148;  // SM count of the device, read at preparation
+  int k1_per_sm = 1;  // resident activation-kernel CTAs per SM (format, rank padding), read at prepare / attach
   svdq_config cfg{};
-  int K = 0, N = 0, N_pad = 0, rank = 0, RP = 0;
+  int K = 0, N = 0, N_pad = 0;
+  int rank = 0, RP = 0;  // branch rank (base + attached adapters) and its padding to a multiple of 32 (0 when empty)
   int fmt = 0;
   float g_x = 1.f, g_w = 1.f, gxgw = 1.f, t_scale = 1.f, denom = 6.f;
   float* s = nullptr;
   float* inv_s = nullptr;
-  __nv_bfloat16* L1T = nullptr;  // [RP, K]
-  __nv_bfloat16* L2T = nullptr;  // [N_pad, RP]
+  // The branch as blocks of columns: the base factors (rank base_rank) and one
+  // block per occupied adapter slot, each as F [K, r] and G [r, N] (bf16).
+  int base_rank = 0;
+  __nv_bfloat16* base_F = nullptr;  // L1 [K, base_rank]
+  __nv_bfloat16* base_G = nullptr;  // L2 [base_rank, N]
+  struct Adapter {
+    int rank = 0;  // 0: slot free
+    __nv_bfloat16* F = nullptr;  // bf16(diag(s) A) [K, rank]
+    __nv_bfloat16* G = nullptr;  // bf16(scale B) [rank, N]
+  } adapters[kMaxAdapters];
+  int col_start[kMaxAdapters + 1] = {};  // slot s owns branch columns [col_start[s], col_start[s+1])
+  // ... assembled in slot order into the layouts the kernels read:
+  __nv_bfloat16* L1T = nullptr;    // [RP, K]  canonical L1'^T
+  __nv_bfloat16* L1sTh = nullptr;  // [RP, K]  bf16 hi of fp32(inv_s[k] L1'[k, j])
+  __nv_bfloat16* L1sTl = nullptr;  // [RP, K]  bf16 lo of the same
+  __nv_bfloat16* L2T = nullptr;    // [N_pad, RP] canonical L2'^T
   __nv_bfloat16* bias = nullptr; // [N_pad], zero beyond N
   uint8_t* wcodes = nullptr;     // INT4 [N_pad, K] E4M3 bytes; NVFP4 [N_pad, K/2]
   void* wscales = nullptr;       // INT4 float [K/64][N_pad]; NVFP4 atoms [N_pad/128][K/64][512]
   int* status = nullptr;         // device status word
   int* k1_counters = nullptr;    // activation-kernel arrival counters per 128-row block (zero between launches)
-  CUtensorMap map_b{}, map_l2{}, map_l1t{};
+  CUtensorMap map_b{}, map_l2{}, map_l1h{}, map_l1l{};
   MapCache<8> ws_maps;  // (workspace, M) -> activation codes map (a), T map (b)
   MapCache<8> x_maps;   // (X, M) -> X map (a)
 };
@@ -143,10 +160,10 @@ WsLayout ws_layout(const svdq_layer* h, int M) {
                                                 : static_cast<size_t>(w.M_pad / 128) * (h->K / 64) * 512;
   w.codes = 0;
   w.scales = align256(cbytes);
-  w.split = act_quant_split(w.M_pad, h->K, h->fmt, h->RP, h->sms);
+  w.split = act_quant_split(w.M_pad, h->K, h->k1_per_sm, h->sms);
   w.T = w.scales + align256(sbytes);
   w.Tpart = w.T + align256(static_cast<size_t>(w.M_pad) * h->RP * 2);
-  const size_t part = w.split > 1 ? static_cast<size_t>(w.split) * w.M_pad * h->RP * 4 : 0;
+  const size_t part = w.split > 1 && h->RP > 0 ? static_cast<size_t>(w.split) * w.M_pad * h->RP * 4 : 0;
   w.total = w.Tpart + align256(part);
   return w;
 }
@@ -165,17 +182,32 @@ svdq_status check_cfg(const svdq_config* cfg) {
   if (!cfg) return fail(SVDQ_ERR_INVALID_ARG, "cfg is NULL");
   if (cfg->K <= 0 || cfg->K % 128) return fail(SVDQ_ERR_INVALID_ARG, "K must be a positive multiple of 128");
   if (cfg->N <= 0 || cfg->N % 16) return fail(SVDQ_ERR_INVALID_ARG, "N must be a positive multiple of 16");
-  if (cfg->rank < 1 || cfg->rank > 256) return fail(SVDQ_ERR_INVALID_ARG, "rank must be in [1, 256]");
+  if (cfg->rank < 0 || cfg->rank > 256) return fail(SVDQ_ERR_INVALID_ARG, "rank must be in [0, 256]");
   if (cfg->rank > std::min(cfg->K, cfg->N)) return fail(SVDQ_ERR_INVALID_ARG, "rank exceeds min(K, N)");
   if (!(cfg->alpha >= 0.f && cfg->alpha <= 1.f)) return fail(SVDQ_ERR_INVALID_ARG, "alpha must be in [0, 1]");
   if (!(cfg->s_min > 0.f) || !std::isfinite(cfg->s_min)) return fail(SVDQ_ERR_INVALID_ARG, "s_min must be > 0");
   if (cfg->fmt != SVDQ_INT4_G64 && cfg->fmt != SVDQ_NVFP4_G16) return fail(SVDQ_ERR_INVALID_ARG, "unknown format");
+  if (cfg->flags & ~static_cast<unsigned>(SVDQ_NO_SMOOTHING)) return fail(SVDQ_ERR_INVALID_ARG, "unknown flags");
   return SVDQ_OK;
+}
+
+// Test hook (svdq_debug_fail_allocation): the library's device allocation
+// with this index (counting from the hook's call) fails as if the device were
+// out of memory; -1 disables it.
+std::atomic<long long> g_fail_alloc_at{-1};
+
+bool injected_alloc_failure() {
+  long long v = g_fail_alloc_at.load(std::memory_order_relaxed);
+  while (v >= 0) {
+    if (g_fail_alloc_at.compare_exchange_weak(v, v - 1, std::memory_order_relaxed)) return v == 0;
+  }
+  return false;
 }
 
 template <class T>
 svdq_status dalloc(T** p, size_t bytes) {
   *p = nullptr;
+  if (injected_alloc_failure()) return fail(SVDQ_ERR_OOM, "device allocation failed (injected by the test hook)");
   if (cudaMalloc(reinterpret_cast<void**>(p), std::max<size_t>(bytes, 256)) != cudaSuccess) {
     cudaGetLastError();
     return fail(SVDQ_ERR_OOM, "cudaMalloc of " + std::to_string(bytes) + " bytes failed");
@@ -187,7 +219,15 @@ void free_layer(svdq_layer* h) {
   if (!h) return;
   cudaFree(h->s);
   cudaFree(h->inv_s);
+  cudaFree(h->base_F);
+  cudaFree(h->base_G);
+  for (auto& a : h->adapters) {
+    cudaFree(a.F);
+    cudaFree(a.G);
+  }
   cudaFree(h->L1T);
+  cudaFree(h->L1sTh);
+  cudaFree(h->L1sTl);
   cudaFree(h->L2T);
   cudaFree(h->bias);
   cudaFree(h->wcodes);
@@ -203,12 +243,19 @@ svdq_status build_static_maps(svdq_layer* h) {
   if (!make_map(&h->map_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, row, h->N_pad, row, 128, kWeightBoxRows,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (weight codes) failed");
-  if (!make_map(&h->map_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->L2T, h->RP, h->N_pad, static_cast<uint64_t>(h->RP) * 2,
-                32, kWeightBoxRows, CU_TENSOR_MAP_SWIZZLE_64B))
-    return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (L2) failed");
-  if (!make_map(&h->map_l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->L1T, h->K, h->RP, static_cast<uint64_t>(h->K) * 2, 64,
-                h->RP, CU_TENSOR_MAP_SWIZZLE_128B))
-    return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (L1) failed");
+  h->map_l2 = CUtensorMap{};
+  h->map_l1h = CUtensorMap{};
+  h->map_l1l = CUtensorMap{};
+  if (h->RP > 0) {
+    if (!make_map(&h->map_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->L2T, h->RP, h->N_pad,
+                  static_cast<uint64_t>(h->RP) * 2, 32, kWeightBoxRows, CU_TENSOR_MAP_SWIZZLE_64B))
+      return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (L2) failed");
+    if (!make_map(&h->map_l1h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->L1sTh, h->K, h->RP, static_cast<uint64_t>(h->K) * 2,
+                  64, h->RP, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&h->map_l1l, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->L1sTl, h->K, h->RP, static_cast<uint64_t>(h->K) * 2,
+                  64, h->RP, CU_TENSOR_MAP_SWIZZLE_128B))
+      return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (L1) failed");
+  }
   h->ws_maps.clear();
   h->x_maps.clear();
   return SVDQ_OK;
@@ -216,13 +263,18 @@ svdq_status build_static_maps(svdq_layer* h) {
 
 // Host part of eq. 2 (float64, one rounding to float32), plus the NVFP4 static
 // activation tensor scale.
-void smoothing_host(const std::vector<float>& a, const std::vector<float>& w, float alpha, float s_min,
+void smoothing_host(const std::vector<float>& a, const std::vector<float>& w, float alpha, float s_min, bool smooth,
                     std::vector<float>& s, std::vector<float>& inv_s) {
   const size_t K = a.size();
   s.resize(K);
   inv_s.resize(K);
   for (size_t k = 0; k < K; ++k) {
     double sk;
+    if (!smooth) {  // the no-smoothing ablation: s = 1 for every channel
+      s[k] = 1.0f;
+      inv_s[k] = 1.0f;
+      continue;
+    }
     if (a[k] == 0.f || w[k] == 0.f) {
       sk = 1.0;
     } else if (alpha == 0.5f) {
@@ -243,6 +295,61 @@ float nvfp4_tensor_scale_host(float amax) {
   return amax / d;
 }
 
+// (Re)builds the kernel layouts of the branch from its blocks (the base
+// factors, then the occupied adapter slots in slot order) into new buffers,
+// and swaps them in only when everything succeeded: on failure the layer is
+// unchanged. Synchronizes `st` before freeing the previous buffers.
+svdq_status assemble_branch(svdq_layer* h, cudaStream_t st) {
+  int cs[kMaxAdapters + 1];
+  cs[0] = h->base_rank;
+  for (int a = 0; a < kMaxAdapters; ++a) cs[a + 1] = cs[a] + h->adapters[a].rank;
+  const int rank = cs[kMaxAdapters];
+  if (rank > 256) return fail(SVDQ_ERR_INVALID_ARG, "branch rank (base + adapters) exceeds 256");
+  const int RP = round_up(rank, 32);
+  __nv_bfloat16 *L1T = nullptr, *L1sTh = nullptr, *L1sTl = nullptr, *L2T = nullptr;
+  auto drop = [&] {
+    cudaFree(L1T);
+    cudaFree(L1sTh);
+    cudaFree(L1sTl);
+    cudaFree(L2T);
+  };
+  if (RP > 0) {
+    const size_t l1 = static_cast<size_t>(RP) * h->K * 2, l2 = static_cast<size_t>(h->N_pad) * RP * 2;
+    svdq_status e;
+    if ((e = dalloc(&L1T, l1)) || (e = dalloc(&L1sTh, l1)) || (e = dalloc(&L1sTl, l1)) || (e = dalloc(&L2T, l2)))
+      return drop(), e;
+    cudaError_t ce = cudaMemsetAsync(L1T, 0, l1, st);
+    if (ce == cudaSuccess) ce = cudaMemsetAsync(L1sTh, 0, l1, st);
+    if (ce == cudaSuccess) ce = cudaMemsetAsync(L1sTl, 0, l1, st);
+    if (ce == cudaSuccess) ce = cudaMemsetAsync(L2T, 0, l2, st);
+    if (ce == cudaSuccess && h->base_rank > 0)
+      ce = launch_assemble_block(h->base_F, h->base_G, h->base_rank, 0, h->K, h->N, RP, h->inv_s, L1T, L1sTh, L1sTl,
+                                 L2T, st);
+    for (int a = 0; a < kMaxAdapters && ce == cudaSuccess; ++a)
+      if (h->adapters[a].rank > 0)
+        ce = launch_assemble_block(h->adapters[a].F, h->adapters[a].G, h->adapters[a].rank, cs[a], h->K, h->N, RP,
+                                   h->inv_s, L1T, L1sTh, L1sTl, L2T, st);
+    if (ce == cudaSuccess) ce = cudaStreamSynchronize(st);
+    if (ce != cudaSuccess) return drop(), fail(SVDQ_ERR_CUDA, std::string("branch assembly: ") + cudaGetErrorString(ce));
+  } else {
+    cudaError_t ce = cudaStreamSynchronize(st);  // earlier work on the old buffers is done before they go
+    if (ce != cudaSuccess) return fail(SVDQ_ERR_CUDA, cudaGetErrorString(ce));
+  }
+  cudaFree(h->L1T);
+  cudaFree(h->L1sTh);
+  cudaFree(h->L1sTl);
+  cudaFree(h->L2T);
+  h->L1T = L1T;
+  h->L1sTh = L1sTh;
+  h->L1sTl = L1sTl;
+  h->L2T = L2T;
+  h->rank = rank;
+  h->RP = RP;
+  for (int a = 0; a <= kMaxAdapters; ++a) h->col_start[a] = cs[a];
+  h->k1_per_sm = act_quant_resident(h->fmt, h->RP);
+  return build_static_maps(h);
+}
+
 // Steps shared by both prepare entry points once L1 [K, rank] and L2 [rank, N]
 // (bf16, device) exist: residual, quantization, branch layout.
 svdq_status finish_prepare(svdq_layer* h, const float* W_hat, const __nv_bfloat16* L1, const __nv_bfloat16* L2,
@@ -252,7 +359,7 @@ svdq_status finish_prepare(svdq_layer* h, const float* W_hat, const __nv_bfloat1
   svdq_status e = dalloc(&R, static_cast<size_t>(K) * N * 4);
   if (e) return e;
   auto cleanup = [&] { cudaFree(R); };
-  if (launch_residual(W_hat, L1, L2, K, N, h->rank, R, st) != cudaSuccess) {
+  if (launch_residual(W_hat, L1, L2, K, N, h->base_rank, R, st) != cudaSuccess) {
     cleanup();
     return fail(SVDQ_ERR_CUDA, "residual kernel launch failed");
   }
@@ -287,11 +394,14 @@ svdq_status finish_prepare(svdq_layer* h, const float* W_hat, const __nv_bfloat1
     if (ce != cudaSuccess) return cleanup(), fail(SVDQ_ERR_CUDA, cudaGetErrorString(ce));
     h->g_w = gw;
   }
-  // branch buffers
-  if ((e = dalloc(&h->L1T, static_cast<size_t>(h->RP) * K * 2))) return cleanup(), e;
-  if ((e = dalloc(&h->L2T, static_cast<size_t>(h->N_pad) * h->RP * 2))) return cleanup(), e;
-  if (launch_build_branch(L1, L2, K, N, h->rank, h->RP, h->N_pad, h->L1T, h->L2T, st) != cudaSuccess)
-    return cleanup(), fail(SVDQ_ERR_CUDA, "branch layout launch failed");
+  // the base block of the branch: the layer keeps its own copy of L1, L2
+  if (h->base_rank > 0) {
+    const size_t f = static_cast<size_t>(K) * h->base_rank * 2, g = static_cast<size_t>(h->base_rank) * N * 2;
+    if ((e = dalloc(&h->base_F, f)) || (e = dalloc(&h->base_G, g))) return cleanup(), e;
+    cudaError_t ce = cudaMemcpyAsync(h->base_F, L1, f, cudaMemcpyDeviceToDevice, st);
+    if (ce == cudaSuccess) ce = cudaMemcpyAsync(h->base_G, L2, g, cudaMemcpyDeviceToDevice, st);
+    if (ce != cudaSuccess) return cleanup(), fail(SVDQ_ERR_CUDA, cudaGetErrorString(ce));
+  }
   cudaError_t ce = cudaStreamSynchronize(st);
   cleanup();
   if (ce != cudaSuccess) return fail(SVDQ_ERR_CUDA, cudaGetErrorString(ce));
@@ -302,18 +412,19 @@ svdq_status finish_prepare(svdq_layer* h, const float* W_hat, const __nv_bfloat1
     h->gxgw = 1.f;
     h->t_scale = 1.f;
   }
-  return build_static_maps(h);
+  return assemble_branch(h, st);
 }
 
 // Steps 1 (statistics, eq. 2) and the migration of eq. 1.
 svdq_status start_prepare(const svdq_config* cfg, const void* W, const void* bias, const float* act_absmax,
                           cudaStream_t st, svdq_layer** out_h, float** W_hat_out) {
   svdq_status e;
-  if ((e = check_device())) return e;
+  // arguments first: a bad call is refused before the device is touched
   if ((e = check_cfg(cfg))) return e;
   if (!W || !act_absmax) return fail(SVDQ_ERR_INVALID_ARG, "W and act_absmax must not be NULL");
   if (!aligned16(W) || (bias && !aligned16(bias)) || !aligned16(act_absmax))
     return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if ((e = check_device())) return e;
   svdq_layer* h = new svdq_layer();
   cudaGetDevice(&h->device);
   if (cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess || h->sms < 1) {
@@ -324,8 +435,7 @@ svdq_status start_prepare(const svdq_config* cfg, const void* W, const void* bia
   h->K = cfg->K;
   h->N = cfg->N;
   h->N_pad = round_up(cfg->N, kNPad);
-  h->rank = cfg->rank;
-  h->RP = round_up(cfg->rank, 32);
+  h->base_rank = cfg->rank;
   h->fmt = cfg->fmt;
   const int K = h->K, N = h->N;
   auto bail = [&](svdq_status s) {
@@ -354,7 +464,7 @@ svdq_status start_prepare(const svdq_config* cfg, const void* W, const void* bia
   if (ce != cudaSuccess) return bail(fail(SVDQ_ERR_CUDA, cudaGetErrorString(ce)));
   for (int k = 0; k < K; ++k)
     if (!(a[k] >= 0.f) || !std::isfinite(a[k])) return bail(fail(SVDQ_ERR_INVALID_ARG, "act_absmax must be finite and >= 0"));
-  smoothing_host(a, w, cfg->alpha, cfg->s_min, s, inv_s);
+  smoothing_host(a, w, cfg->alpha, cfg->s_min, (cfg->flags & SVDQ_NO_SMOOTHING) == 0, s, inv_s);
   if (cfg->fmt == SVDQ_NVFP4_G16) {
     float amax_x = 0.f;
     for (int k = 0; k < K; ++k) {
@@ -425,7 +535,7 @@ svdq_status svd_factors(svdq_layer* h, const float* W_hat, __nv_bfloat16* L1, __
   if (ce == cudaSuccess) ce = cudaStreamSynchronize(st);
   if (ce != cudaSuccess) return cleanup(), fail(SVDQ_ERR_CUDA, cudaGetErrorString(ce));
   if (hinfo != 0) return cleanup(), fail(SVDQ_ERR_NUMERIC, "gesvd did not converge (info=" + std::to_string(hinfo) + ")");
-  if (launch_factors_from_svd(U, S, VT, K, N, h->rank, wt, m, n, L1, L2, st) != cudaSuccess)
+  if (launch_factors_from_svd(U, S, VT, K, N, h->base_rank, wt, m, n, L1, L2, st) != cudaSuccess)
     return cleanup(), fail(SVDQ_ERR_CUDA, "factor kernel launch failed");
   ce = cudaStreamSynchronize(st);
   cleanup();
@@ -434,7 +544,7 @@ svdq_status svd_factors(svdq_layer* h, const float* W_hat, __nv_bfloat16* L1, __
 }
 
 svdq_status launch_k1(svdq_layer* h, const void* X, int M, uint8_t* codes, void* scales, __nv_bfloat16* T,
-                      float* Tpart, const WsLayout& w, cudaStream_t st) {
+                      float* Tpart, const WsLayout& w, const uint32_t* row_mask, cudaStream_t st) {
   if (w.M_pad / 128 > kMaxRowBlocks) return fail(SVDQ_ERR_INVALID_ARG, "M exceeds the supported row count");
   ActQuantParams p{};
   p.split = w.split;
@@ -445,7 +555,6 @@ svdq_status launch_k1(svdq_layer* h, const void* X, int M, uint8_t* codes, void*
   p.K = h->K;
   p.M_pad = round_up(M, 128);
   p.inv_s = h->inv_s;
-  p.L1T = h->L1T;
   p.codes = codes;
   p.scales = scales;
   p.T = T;
@@ -453,6 +562,8 @@ svdq_status launch_k1(svdq_layer* h, const void* X, int M, uint8_t* codes, void*
   p.denom = h->denom;
   p.t_scale = h->t_scale;
   p.status = h->status;
+  p.row_mask = row_mask;
+  for (int a = 0; a <= kMaxAdapters; ++a) p.col_start[a] = h->col_start[a];
   ActQuantMaps maps;
   auto* xe = h->x_maps.find(X, M);
   if (!xe) {
@@ -464,7 +575,8 @@ svdq_status launch_k1(svdq_layer* h, const void* X, int M, uint8_t* codes, void*
     }
   }
   maps.x = xe->a;
-  maps.l1t = h->map_l1t;
+  maps.l1h = h->map_l1h;
+  maps.l1l = h->map_l1l;
   cudaError_t e = launch_act_quant(p, maps, h->fmt, h->RP, st);
   if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("activation kernel: ") + cudaGetErrorString(e));
   return SVDQ_OK;
@@ -472,6 +584,19 @@ svdq_status launch_k1(svdq_layer* h, const void* X, int M, uint8_t* codes, void*
 
 svdq_status check_layer(svdq_layer* h) {
   if (!h) return fail(SVDQ_ERR_INVALID_ARG, "layer is NULL");
+  return SVDQ_OK;
+}
+
+// Calls that launch kernels on a layer's buffers must run with the layer's
+// device current: its weights, tensor maps and scratch live there.
+svdq_status check_layer_device(svdq_layer* h) {
+  if (check_layer(h)) return SVDQ_ERR_INVALID_ARG;
+  int dev = -1;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  if (dev != h->device)
+    return fail(SVDQ_ERR_INVALID_ARG, "the current device (" + std::to_string(dev) + ") is not the layer's device (" +
+                                          std::to_string(h->device) + ")");
   return SVDQ_OK;
 }
 
@@ -483,6 +608,7 @@ const char* svdq_last_error(void) { return g_last_error.c_str(); }
 
 svdq_status svdq_calibrate_absmax(const void* X, int M, int K, float* absmax_inout, void* stream) {
   if (!X || !absmax_inout || M < 1 || K < 1) return fail(SVDQ_ERR_INVALID_ARG, "bad calibration arguments");
+  if (!aligned16(X) || !aligned16(absmax_inout)) return fail(SVDQ_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   if (launch_absmax_cols(static_cast<const __nv_bfloat16*>(X), M, K, absmax_inout, static_cast<cudaStream_t>(stream)) !=
       cudaSuccess)
     return fail(SVDQ_ERR_CUDA, "calibration kernel launch failed");
@@ -499,9 +625,13 @@ svdq_status svdq_prepare_weights(const svdq_config* cfg, const void* W, const vo
   svdq_status e = start_prepare(cfg, W, bias, act_absmax, st, &h, &W_hat);
   if (e) return e;
   __nv_bfloat16 *L1 = nullptr, *L2 = nullptr;
-  if ((e = dalloc(&L1, static_cast<size_t>(h->K) * h->rank * 2)) ||
-      (e = dalloc(&L2, static_cast<size_t>(h->rank) * h->N * 2)) || (e = svd_factors(h, W_hat, L1, L2, st)) ||
-      (e = finish_prepare(h, W_hat, L1, L2, st))) {
+  // rank 0 (smoothing only, no branch) needs no decomposition
+  if (h->base_rank > 0 && ((e = dalloc(&L1, static_cast<size_t>(h->K) * h->base_rank * 2)) ||
+                           (e = dalloc(&L2, static_cast<size_t>(h->base_rank) * h->N * 2)) ||
+                           (e = svd_factors(h, W_hat, L1, L2, st))))
+    ;
+  if (e == SVDQ_OK) e = finish_prepare(h, W_hat, L1, L2, st);
+  if (e) {
     cudaFree(L1);
     cudaFree(L2);
     cudaFree(W_hat);
@@ -520,7 +650,9 @@ svdq_status svdq_prepare_weights_with_factors(const svdq_config* cfg, const void
                                               svdq_layer_t* out) {
   if (!out) return fail(SVDQ_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
-  if (!L1 || !L2) return fail(SVDQ_ERR_INVALID_ARG, "L1 and L2 must not be NULL");
+  if (cfg && cfg->rank > 0 && (!L1 || !L2)) return fail(SVDQ_ERR_INVALID_ARG, "L1 and L2 must not be NULL");
+  if ((L1 && !aligned16(L1)) || (L2 && !aligned16(L2)))
+    return fail(SVDQ_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   svdq_layer* h = nullptr;
   float* W_hat = nullptr;
@@ -548,13 +680,16 @@ svdq_status svdq_workspace_size(svdq_layer_t h, int M, size_t* bytes) {
 namespace {
 
 svdq_status forward_impl(svdq_layer* h, const void* X, int M, void* Y, void* workspace, size_t ws_bytes,
-                         void* stream, void* const* events) {
+                         const uint32_t* row_mask, void* stream, void* const* events) {
   if (check_layer(h)) return SVDQ_ERR_INVALID_ARG;
   if (!X || !Y || !workspace || M < 1) return fail(SVDQ_ERR_INVALID_ARG, "NULL pointer or M < 1");
   if (!aligned16(X) || !aligned16(Y) || (reinterpret_cast<uintptr_t>(workspace) & 255))
     return fail(SVDQ_ERR_INVALID_ARG, "X/Y must be 16-byte and the workspace 256-byte aligned");
+  if (row_mask && (reinterpret_cast<uintptr_t>(row_mask) & 3))
+    return fail(SVDQ_ERR_INVALID_ARG, "row_mask must be 4-byte aligned");
   const WsLayout w = ws_layout(h, M);
   if (ws_bytes < w.total) return fail(SVDQ_ERR_INVALID_ARG, "workspace too small");
+  if (svdq_status e = check_layer_device(h)) return e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(workspace);
   uint8_t* codes = base + w.codes;
@@ -562,7 +697,7 @@ svdq_status forward_impl(svdq_layer* h, const void* X, int M, void* Y, void* wor
   __nv_bfloat16* T = reinterpret_cast<__nv_bfloat16*>(base + w.T);
   if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[0]), st));
   float* Tpart = reinterpret_cast<float*>(base + w.Tpart);
-  svdq_status e = launch_k1(h, X, M, codes, scales, T, Tpart, w, st);
+  svdq_status e = launch_k1(h, X, M, codes, scales, T, Tpart, w, row_mask, st);
   if (e) return e;
   if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[1]), st));
   auto* we = h->ws_maps.find(workspace, M);
@@ -570,10 +705,11 @@ svdq_status forward_impl(svdq_layer* h, const void* X, int M, void* Y, void* wor
     we = h->ws_maps.insert(workspace, M);
     const bool i4 = h->fmt == SVDQ_INT4_G64;
     const uint64_t row = i4 ? h->K : h->K / 2;
+    we->b = CUtensorMap{};
     if (!make_map(&we->a, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, row, w.M_pad, row, 128, kActBoxRows,
                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&we->b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, h->RP, w.M_pad, static_cast<uint64_t>(h->RP) * 2, 32,
-                  128, CU_TENSOR_MAP_SWIZZLE_64B)) {
+        (h->RP > 0 && !make_map(&we->b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, h->RP, w.M_pad,
+                                static_cast<uint64_t>(h->RP) * 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))) {
       we->key = nullptr;
       return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (activations) failed");
     }
@@ -608,66 +744,95 @@ extern "C" {
 
 svdq_status svdq_linear_forward(svdq_layer_t h, const void* X, int M, void* Y, void* workspace, size_t ws_bytes,
                                 void* stream) {
-  return forward_impl(h, X, M, Y, workspace, ws_bytes, stream, nullptr);
+  return forward_impl(h, X, M, Y, workspace, ws_bytes, nullptr, stream, nullptr);
+}
+
+svdq_status svdq_linear_forward_masked(svdq_layer_t h, const void* X, int M, void* Y, void* workspace,
+                                       size_t ws_bytes, const uint32_t* row_adapter_mask, void* stream) {
+  if (!row_adapter_mask) return fail(SVDQ_ERR_INVALID_ARG, "row_adapter_mask is NULL (use svdq_linear_forward)");
+  return forward_impl(h, X, M, Y, workspace, ws_bytes, row_adapter_mask, stream, nullptr);
 }
 
 svdq_status svdq_linear_forward_profiled(svdq_layer_t h, const void* X, int M, void* Y, void* workspace,
                                          size_t ws_bytes, void* stream, void* const* events) {
   if (!events || !events[0] || !events[1] || !events[2]) return fail(SVDQ_ERR_INVALID_ARG, "three events needed");
-  return forward_impl(h, X, M, Y, workspace, ws_bytes, stream, events);
+  return forward_impl(h, X, M, Y, workspace, ws_bytes, nullptr, stream, events);
 }
 
 svdq_status svdq_quantize_activations(svdq_layer_t h, const void* X, int M, void* codes, void* scales, void* T,
                                       void* stream) {
   if (check_layer(h)) return SVDQ_ERR_INVALID_ARG;
-  if (!X || !codes || !scales || !T || M < 1) return fail(SVDQ_ERR_INVALID_ARG, "NULL pointer or M < 1");
-  if (!aligned16(X) || !aligned16(codes) || !aligned16(scales) || !aligned16(T))
+  if (!X || !codes || !scales || (!T && h->RP > 0) || M < 1) return fail(SVDQ_ERR_INVALID_ARG, "NULL pointer or M < 1");
+  if (!aligned16(X) || !aligned16(codes) || !aligned16(scales) || (T && !aligned16(T)))
     return fail(SVDQ_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (svdq_status e = check_layer_device(h)) return e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const WsLayout w = ws_layout(h, M);
   // float partials over the K shares: a scratch buffer of this call's own
   float* Tpart = nullptr;
-  if (w.split > 1) {
+  if (w.split > 1 && h->RP > 0) {
+    if (injected_alloc_failure()) return fail(SVDQ_ERR_OOM, "device allocation failed (injected by the test hook)");
     cudaError_t ce = cudaMallocAsync(reinterpret_cast<void**>(&Tpart), w.total - w.Tpart, st);
     if (ce != cudaSuccess) return fail(SVDQ_ERR_OOM, std::string("T partials: ") + cudaGetErrorString(ce));
   }
-  svdq_status e = launch_k1(h, X, M, static_cast<uint8_t*>(codes), scales, static_cast<__nv_bfloat16*>(T), Tpart, w, st);
+  svdq_status e =
+      launch_k1(h, X, M, static_cast<uint8_t*>(codes), scales, static_cast<__nv_bfloat16*>(T), Tpart, w, nullptr, st);
   if (Tpart) cudaFreeAsync(Tpart, st);
   return e;
 }
 
-svdq_status svdq_attach_lora(svdq_layer_t h, const void* A, const void* B, int r_l, float scale, void* stream) {
+svdq_status svdq_attach_lora(svdq_layer_t h, const void* A, const void* B, int r_l, float scale, void* stream,
+                             int* slot_out) {
+  if (slot_out) *slot_out = -1;
   if (check_layer(h)) return SVDQ_ERR_INVALID_ARG;
   if (!A || !B || r_l < 1) return fail(SVDQ_ERR_INVALID_ARG, "bad LoRA arguments");
   if (h->rank + r_l > 256) return fail(SVDQ_ERR_INVALID_ARG, "rank + r_l exceeds 256");
   if (!std::isfinite(scale)) return fail(SVDQ_ERR_INVALID_ARG, "scale must be finite");
+  if (!aligned16(A) || !aligned16(B)) return fail(SVDQ_ERR_INVALID_ARG, "A and B must be 16-byte aligned");
+  int slot = -1;
+  for (int a = 0; a < kMaxAdapters && slot < 0; ++a)
+    if (h->adapters[a].rank == 0) slot = a;
+  if (slot < 0) return fail(SVDQ_ERR_INVALID_ARG, "every adapter slot is taken (detach one first)");
+  if (svdq_status e = check_layer_device(h)) return e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int new_rank = h->rank + r_l;
-  const int RP_new = round_up(new_rank, 32);
-  __nv_bfloat16 *L1T = nullptr, *L2T = nullptr;
+  svdq_layer::Adapter ad;
+  ad.rank = r_l;
   svdq_status e;
-  if ((e = dalloc(&L1T, static_cast<size_t>(RP_new) * h->K * 2))) return e;
-  if ((e = dalloc(&L2T, static_cast<size_t>(h->N_pad) * RP_new * 2))) return cudaFree(L1T), e;
-  if (launch_lora_concat(h->L1T, h->L2T, h->K, h->N, h->N_pad, h->rank, h->RP, h->s,
-                         static_cast<const __nv_bfloat16*>(A), static_cast<const __nv_bfloat16*>(B), r_l, scale, RP_new,
-                         L1T, L2T, st) != cudaSuccess) {
-    cudaFree(L1T);
-    cudaFree(L2T);
-    return fail(SVDQ_ERR_CUDA, "LoRA concat launch failed");
+  if ((e = dalloc(&ad.F, static_cast<size_t>(h->K) * r_l * 2))) return e;
+  if ((e = dalloc(&ad.G, static_cast<size_t>(r_l) * h->N * 2))) return cudaFree(ad.F), e;
+  if (launch_lora_factors(static_cast<const __nv_bfloat16*>(A), static_cast<const __nv_bfloat16*>(B), h->K, h->N, r_l,
+                          scale, h->s, ad.F, ad.G, st) != cudaSuccess) {
+    cudaFree(ad.F);
+    cudaFree(ad.G);
+    return fail(SVDQ_ERR_CUDA, "LoRA factor launch failed");
   }
-  cudaError_t ce = cudaStreamSynchronize(st);
-  if (ce != cudaSuccess) {
-    cudaFree(L1T);
-    cudaFree(L2T);
-    return fail(SVDQ_ERR_CUDA, cudaGetErrorString(ce));
+  h->adapters[slot] = ad;
+  if ((e = assemble_branch(h, st))) {
+    cudaStreamSynchronize(st);
+    cudaFree(ad.F);
+    cudaFree(ad.G);
+    h->adapters[slot] = svdq_layer::Adapter{};
+    return e;
   }
-  cudaFree(h->L1T);
-  cudaFree(h->L2T);
-  h->L1T = L1T;
-  h->L2T = L2T;
-  h->rank = new_rank;
-  h->RP = RP_new;
-  return build_static_maps(h);
+  if (slot_out) *slot_out = slot;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_detach_lora(svdq_layer_t h, int slot, void* stream) {
+  if (check_layer(h)) return SVDQ_ERR_INVALID_ARG;
+  if (slot < 0 || slot >= kMaxAdapters || h->adapters[slot].rank == 0)
+    return fail(SVDQ_ERR_INVALID_ARG, "no adapter in slot " + std::to_string(slot));
+  if (svdq_status e = check_layer_device(h)) return e;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const svdq_layer::Adapter ad = h->adapters[slot];
+  h->adapters[slot] = svdq_layer::Adapter{};
+  if (svdq_status e = assemble_branch(h, st)) {
+    h->adapters[slot] = ad;  // nothing was swapped: the layer keeps the adapter
+    return e;
+  }
+  cudaFree(ad.F);
+  cudaFree(ad.G);
+  return SVDQ_OK;
 }
 
 svdq_status svdq_layer_get_info(svdq_layer_t h, svdq_layer_info* info) {
@@ -677,6 +842,14 @@ svdq_status svdq_layer_get_info(svdq_layer_t h, svdq_layer_info* info) {
   info->N = h->N;
   info->rank = h->rank;
   info->rank_pad = h->RP;
+  info->base_rank = h->base_rank;
+  info->flags = h->cfg.flags;
+  info->adapter_slots = 0;
+  for (int a = 0; a < kMaxAdapters; ++a) {
+    if (h->adapters[a].rank) info->adapter_slots |= 1u << a;
+    info->adapter_col_start[a] = h->col_start[a];
+  }
+  info->adapter_col_start[kMaxAdapters] = h->col_start[kMaxAdapters];
   info->fmt = h->fmt;
   info->alpha = h->cfg.alpha;
   info->g_x = h->g_x;
@@ -730,8 +903,10 @@ svdq_status svdq_export_weights(svdq_layer_t h, void* blob, size_t* bytes, void*
   CUDA_TRY(cudaMemcpyAsync(b + hd.off_s, h->s, K * 4, cudaMemcpyDeviceToHost, st));
   CUDA_TRY(cudaMemcpyAsync(b + hd.off_inv_s, h->inv_s, K * 4, cudaMemcpyDeviceToHost, st));
   CUDA_TRY(cudaMemcpyAsync(b + hd.off_bias, h->bias, N * 2, cudaMemcpyDeviceToHost, st));
-  CUDA_TRY(cudaMemcpyAsync(l1t.data(), h->L1T, l1t.size() * 2, cudaMemcpyDeviceToHost, st));
-  CUDA_TRY(cudaMemcpyAsync(l2t.data(), h->L2T, l2t.size() * 2, cudaMemcpyDeviceToHost, st));
+  if (h->RP > 0) {
+    CUDA_TRY(cudaMemcpyAsync(l1t.data(), h->L1T, l1t.size() * 2, cudaMemcpyDeviceToHost, st));
+    CUDA_TRY(cudaMemcpyAsync(l2t.data(), h->L2T, l2t.size() * 2, cudaMemcpyDeviceToHost, st));
+  }
   CUDA_TRY(cudaMemcpyAsync(codes.data(), h->wcodes, cbytes, cudaMemcpyDeviceToHost, st));
   CUDA_TRY(cudaMemcpyAsync(scales.data(), h->wscales, sbytes, cudaMemcpyDeviceToHost, st));
   CUDA_TRY(cudaStreamSynchronize(st));
@@ -801,6 +976,8 @@ svdq_status svdq_destroy(svdq_layer_t h) {
   free_layer(h);
   return SVDQ_OK;
 }
+
+void svdq_debug_fail_allocation(long long index) { g_fail_alloc_at.store(index < 0 ? -1 : index); }
 
 svdq_status svdq_selftest_bounded_wait(unsigned long long limit_ns, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);

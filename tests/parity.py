@@ -46,9 +46,11 @@ class Case:
 
 
 def oracle_case(layer: workloads.Layer) -> Case:
+    """The oracle on the layer's inputs; layer.meta["smooth"] = False selects
+    the no-smoothing ablation (rank 0, the smoothing-only one, is layer.rank)."""
     X, W, b = workloads.to_f64(layer.X), workloads.to_f64(layer.W), workloads.to_f64(layer.bias)
     a = S.calibrate_absmax(X)
-    p = S.prepare(W, b, a, layer.fmt, layer.alpha, layer.rank)
+    p = S.prepare(W, b, a, layer.fmt, layer.alpha, layer.rank, smooth=layer.meta.get("smooth", True))
     return Case(layer, X, W, b, a, p, S.forward(p, X))
 
 
@@ -59,7 +61,8 @@ def gpu_prepare(case: Case, with_factors: bool = True):
     bias = L.bias.cuda()
     a = torch.from_numpy(case.a).cuda()
     factors = (bf16_tensor(case.p.L1), bf16_tensor(case.p.L2)) if with_factors else None
-    return rq.Layer.prepare(W, bias, a, L.fmt, L.rank, alpha=L.alpha, factors=factors)
+    return rq.Layer.prepare(W, bias, a, L.fmt, L.rank, alpha=L.alpha, factors=factors,
+                            smooth=L.meta.get("smooth", True))
 
 
 def canonical_weight_codes(p: oracle.Prepared) -> np.ndarray:

@@ -69,3 +69,30 @@ def test_workload_names_carry_the_shapes():
     import workloads
     d = bench.workload_desc(1, workloads.config(0))  # any layer list; the name follows the config id
     assert "attention projection" in d
+
+
+def test_peak_follows_the_length_of_the_timed_region():
+    peaks = {"bf16_tflops": 1640.7, "bf16_tflops_sustained": 1376.5}
+    burst, d1 = bench.tensor_peak_for(peaks, "nvfp4_g16", 0.0065)
+    assert burst == pytest.approx(4 * 1640.7) and "burst" in d1
+    sus, d2 = bench.tensor_peak_for(peaks, "nvfp4_g16", 6.5)
+    assert sus == pytest.approx(4 * 1376.5) and "sustained" in d2
+    assert bench.tensor_peak_for(peaks, "int4_g64", 0.003)[0] == pytest.approx(2 * 1640.7)
+
+
+def test_both_arms_emit_the_same_config():
+    import argparse
+
+    import workloads
+    args = argparse.Namespace(config=0, M=0, rank=0, fmt=None)
+    layers = bench.load_layers(args)
+    a, b = bench.config_dict(args, layers), bench.config_dict(args, workloads.config(0))
+    assert a == b and "l2" in a and a["config_id"] == 0
+    n_sets, set_bytes = bench.rotation_sets(layers)
+    assert n_sets * set_bytes > 2 * bench.L2_BYTES
+
+
+def test_default_workload_is_the_nvfp4_mlp_pair():
+    args = bench.parse_args([])
+    assert args.config == 3 and args.gpus == 1 and args.impl == "ours"
+    assert bench.parse_args(["--config", "1"]).config == 1

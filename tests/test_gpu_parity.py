@@ -28,7 +28,17 @@ SMALL = {
     "m1_nvfp4": lambda: workloads.custom(1, 256, 128, 8, workloads.NVFP4_G16, seed=74),
     "rank100_nvfp4": lambda: workloads.custom(300, 512, 256, 100, workloads.NVFP4_G16, seed=75),
     "rank100_int4": lambda: workloads.custom(300, 512, 256, 100, workloads.INT4_G64, seed=76),
+    # ablations: rank 0 (smoothing only, no branch) and no smoothing (s = 1)
+    "rank0_int4": lambda: workloads.custom(260, 512, 384, 0, workloads.INT4_G64, seed=77),
+    "rank0_nvfp4": lambda: workloads.custom(260, 512, 384, 0, workloads.NVFP4_G16, seed=78),
+    "nosmooth_int4": lambda: _no_smoothing(workloads.custom(200, 512, 256, 32, workloads.INT4_G64, seed=79)),
+    "nosmooth_nvfp4": lambda: _no_smoothing(workloads.custom(200, 512, 256, 32, workloads.NVFP4_G16, seed=80)),
 }
+
+
+def _no_smoothing(layer):
+    layer.meta["smooth"] = False
+    return layer
 
 
 def _as_fmt(layer, fmt):
@@ -104,7 +114,7 @@ def test_forward_is_deterministic_and_reuses_workspace(small):
     assert torch.equal(y1, y2)
 
 
-@pytest.mark.parametrize("name", ["cfg0_int4", "ragged_nvfp4", "rank100_int4"])
+@pytest.mark.parametrize("name", ["cfg0_int4", "ragged_nvfp4", "rank100_int4", "rank0_nvfp4", "nosmooth_int4"])
 def test_full_prepare_with_cusolver_svd(name):
     case = oracle_case(SMALL[name]())
     g = gpu_prepare(case, with_factors=False)

@@ -197,16 +197,21 @@ def _bf(x):
     return float(F.bf16_round(np.float64(x)))
 
 
-def _brute_force_layer(X, W, b, a, fmt, rank, L1, L2):
+def _brute_force_layer(X, W, b, a, fmt, rank, L1, L2, smooth=True):
     """Every quantity of a tiny layer recomputed with plain Python loops from
     the definitions (no vectorized oracle code): eq. 2, eq. 1, R = W_hat - L1 L2,
-    the group quantizers, the integer / E2M1 group sums, the branch and the bias."""
+    the group quantizers, the integer / E2M1 group sums, the branch and the bias.
+    smooth=False: s = 1 everywhere (no migration)."""
     K, N = W.shape
     M = X.shape[0]
     s, inv_s = [], []
     for k in range(K):
         wk = max(abs(W[k, n]) for n in range(N))
         ak = float(a[k])
+        if not smooth:
+            s.append(F32(1.0))
+            inv_s.append(F32(1.0))
+            continue
         if ak == 0 or wk == 0:
             sk = 1.0
         else:
@@ -332,3 +337,132 @@ def test_lora_attach_changes_only_the_branch():
     # and, up to bf16 rounding of diag(s) A and scale B, it is the LoRA term scale * X A B
     ref = 0.5 * X @ A @ B
     assert np.linalg.norm(delta - ref) / np.linalg.norm(ref) < 1e-2
+
+
+
+# ------------------------------------------------- ablations of the method
+
+@pytest.mark.parametrize("fmt", workloads.FORMATS)
+@pytest.mark.parametrize("rank,smooth", [(0, True), (2, False), (0, False)])
+def test_tiny_ablation_layers_brute_force(fmt, rank, smooth):
+    """Rank 0 (smoothing only: the SmoothQuant special case of the entry's
+    related terms) and no smoothing (s = 1) recomputed by plain loops."""
+    layer = workloads.custom(3, 128, 8, max(rank, 1), fmt, seed=43, n_outliers=2)
+    X, W, b = workloads.to_f64(layer.X), workloads.to_f64(layer.W), workloads.to_f64(layer.bias)
+    a = S.calibrate_absmax(X)
+    p = S.prepare(W, b, a, fmt, 0.5, rank, smooth=smooth)
+    assert p.L1.shape == (128, rank) and p.L2.shape == (rank, 8)
+    y = S.forward(p, X).Y
+    yb = _brute_force_layer(X, W, b, a, fmt, rank, p.L1, p.L2, smooth=smooth)
+    assert np.allclose(y, yb, rtol=1e-12, atol=1e-12)
+
+
+def test_rank0_residual_is_the_migrated_weight_and_the_branch_is_empty():
+    layer = workloads.custom(16, 128, 64, 1, "nvfp4_g16", seed=44)
+    X, W, b = workloads.to_f64(layer.X), workloads.to_f64(layer.W), workloads.to_f64(layer.bias)
+    p = S.prepare(W, b, S.calibrate_absmax(X), "nvfp4_g16", 0.5, 0)
+    assert np.array_equal(p.R.view(np.uint32), S.migrate_weight(W, p.s).view(np.uint32))
+    r = S.forward(p, X)
+    assert r.T.shape == (16, 0)
+    assert np.array_equal(r.Y, r.main + p.bias[None, :])
+    y = S.forward_unquantized(p, X)  # the equivalence holds without a branch too
+    assert np.linalg.norm(y - (X @ W + b)) / np.linalg.norm(X @ W + b) < 2e-6
+
+
+def test_no_smoothing_leaves_activations_and_weights_as_they_are():
+    layer = workloads.custom(16, 128, 64, 4, "int4_g64", seed=45)
+    X, W, b = workloads.to_f64(layer.X), workloads.to_f64(layer.W), workloads.to_f64(layer.bias)
+    p = S.prepare(W, b, S.calibrate_absmax(X), "int4_g64", 0.5, 4, smooth=False)
+    assert np.all(p.s == 1.0) and np.all(p.inv_s == 1.0)
+    assert np.array_equal(S.smooth_activations(X, p.inv_s), X.astype(F32))
+    y = S.forward_unquantized(p, X)
+    assert np.linalg.norm(y - (X @ W + b)) / np.linalg.norm(X @ W + b) < 2e-6
+
+
+def test_ablation_error_ordering_on_outlier_data():
+    """Diagnostic (abstract; section 2.1): on outlier activations the full
+    method beats smoothing alone, which beats no smoothing, in both formats."""
+    for fmt in workloads.FORMATS:
+        layer = workloads.custom(128, 512, 256, 32, fmt, seed=46, n_outliers=6)
+        X, W, b = workloads.to_f64(layer.X), workloads.to_f64(layer.W), workloads.to_f64(layer.bias)
+        ref = X @ W + b
+        a = S.calibrate_absmax(X)
+        err = lambda p: np.linalg.norm(S.forward(p, X).Y - ref) / np.linalg.norm(ref)
+        full = err(S.prepare(W, b, a, fmt, 0.5, 32))
+        smooth_only = err(S.prepare(W, b, a, fmt, 0.5, 0))
+        naive = err(S.prepare(W, b, a, fmt, 0.5, 0, smooth=False))
+        assert full < smooth_only < naive, (fmt, full, smooth_only, naive)
+
+
+# ------------------------------------------- per-row adapter selection
+
+def test_selected_adapters_follow_their_definition():
+    """Per-row selection against the composition it must equal: all bits set
+    is the layer with both adapters concatenated (attach_lora twice), no bit
+    set is the layer alone, one bit is the layer with that adapter alone."""
+    layer = workloads.custom(12, 128, 64, 4, "nvfp4_g16", seed=52, lora_rank=8)
+    X, W, b = workloads.to_f64(layer.X), workloads.to_f64(layer.W), workloads.to_f64(layer.bias)
+    A0, B0 = workloads.to_f64(layer.lora_A), workloads.to_f64(layer.lora_B)
+    rng = np.random.Generator(np.random.PCG64(53))
+    A1 = F.bf16_round(rng.normal(0, 0.01, (128, 16)))
+    B1 = F.bf16_round(rng.normal(0, 0.01, (16, 64)))
+    p = S.prepare(W, b, S.calibrate_absmax(X), "nvfp4_g16", 0.5, 4)
+    ads = {0: S.lora_factors(p, A0, B0, 0.5), 1: S.lora_factors(p, A1, B1, 2.0)}
+    mask = np.array([0b11, 0b00, 0b01, 0b10] * 3)
+    y = S.forward_selected(p, ads, X, mask)
+    both = S.forward(S.attach_lora(S.attach_lora(p, A0, B0, 0.5), A1, B1, 2.0), X).Y
+    only0 = S.forward(S.attach_lora(p, A0, B0, 0.5), X).Y
+    only1 = S.forward(S.attach_lora(p, A1, B1, 2.0), X).Y
+    base = S.forward(p, X).Y
+    for m in range(12):
+        want = {0b11: both, 0b00: base, 0b01: only0, 0b10: only1}[mask[m]][m]
+        assert np.allclose(y[m], want, rtol=1e-12, atol=1e-13), m
+    assert np.array_equal(y[mask == 0], base[mask == 0])
+    # a planted mistake: slot bits read the wrong way round
+    y_bad = S.forward_selected(p, {0: ads[1], 1: ads[0]}, X, mask)
+    assert not np.allclose(y_bad[mask == 0b01], only0[mask == 0b01], rtol=1e-6)
+
+
+# ------------------------------------------------- the weight-only baseline
+
+def test_weight_only_brute_force():
+    layer = workloads.custom(3, 128, 8, 1, "int4_g64", seed=47)
+    X, W, b = workloads.to_f64(layer.X), workloads.to_f64(layer.W), workloads.to_f64(layer.bias)
+    p = S.prepare_weight_only(W, b)
+    y = S.forward_weight_only(p, X)
+    K, N = W.shape
+    yb = np.zeros((3, N))
+    for n in range(N):
+        w = []
+        for g0 in range(0, K, 64):
+            col = [F32(W[k, n]) for k in range(g0, g0 + 64)]
+            amax = F32(max(abs(float(v)) for v in col))
+            if amax == 0:
+                w += [0.0] * 64
+                continue
+            inv, sc = F32(F32(7.0) / amax), F32(amax / F32(7.0))
+            for v in col:
+                t = float(F32(v * inv))
+                q = min(range(-8, 8), key=lambda c: (abs(t - c), c % 2))
+                w.append(_bf(float(F32(F32(q) * sc))))
+        for m in range(3):
+            yb[m, n] = sum(X[m, k] * w[k] for k in range(K)) + b[n]
+    assert np.allclose(y, yb, rtol=1e-12, atol=1e-12)
+
+
+def test_weight_only_is_exact_on_representable_weights():
+    """Weights that are already integer multiples (|q| <= 7, each group's
+    largest |q| = 7) of a power-of-two group scale quantize without error:
+    the baseline then computes X W + b exactly (every product and partial sum
+    is exact in float64 for these small integers)."""
+    rng = np.random.Generator(np.random.PCG64(48))
+    K, N, M = 256, 16, 5
+    q = rng.integers(-7, 8, size=(K, N))
+    q[::64, :] = 7  # each group of 64 along k reaches amax = 7 * scale
+    scale = 2.0 ** rng.integers(-6, -2, size=(K // 64, N))
+    W = q * np.repeat(scale, 64, axis=0)
+    X = rng.integers(-4, 5, size=(M, K)).astype(np.float64)
+    b = rng.integers(-3, 4, size=N) * 0.125
+    p = S.prepare_weight_only(W, b)
+    assert np.array_equal(S.dequantize_weight_only(p), W.T)
+    assert np.array_equal(S.forward_weight_only(p, X), X @ W + b)

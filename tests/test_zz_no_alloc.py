@@ -76,3 +76,26 @@ def test_noalloc_refuses_a_workspace_beyond_the_scratch():
         assert rel(f64(Y2), case.r.Y) <= Y_TOL
     finally:
         g.close()
+
+
+@pytest.mark.parametrize("fmt", workloads.FORMATS)
+def test_attention_projection_at_rank_128_fits_the_scratch(fmt):
+    """The fixed scratch covers the 4608 x 3072 x 3072 attention projection up
+    to rank 128 in both formats (the activation kernel's K split, which sets
+    the size of its float partials, included)."""
+    import rank_gemm_quantize_b200 as rq
+    M, K, N, r = 4608, 3072, 3072, 128
+    gen = torch.Generator(device="cpu").manual_seed(5)
+    W = (torch.randn(K, N, generator=gen) * 0.02).to(torch.bfloat16).cuda()
+    L1 = (torch.randn(K, r, generator=gen) * 0.02).to(torch.bfloat16).cuda()
+    L2 = (torch.randn(r, N, generator=gen) * 0.02).to(torch.bfloat16).cuda()
+    a = torch.ones(K, dtype=torch.float32, device="cuda")
+    g = rq.Layer.prepare(W, None, a, fmt, r, factors=(L1, L2))
+    try:
+        need = g.workspace_size(M)
+        assert need <= SCRATCH_BYTES, need
+        Y = g.forward_noalloc(torch.zeros(M, K, dtype=torch.bfloat16, device="cuda"))
+        torch.cuda.synchronize()
+        assert int(torch.count_nonzero(Y)) == 0  # zero input, no bias: Y = 0
+    finally:
+        g.close()
