@@ -46,8 +46,17 @@ RATE_VS_BF16 = {"nvfp4_g16": 4.0, "int4_g64": 2.0}  # mxf4nvf4 = 4x bf16; f8f6f4
 TRAFFIC_RECORDS_FILE = os.path.join(ROOT, "profiles", "traffic_records.txt")
 
 
-def workload_desc(cfg: int, layers) -> str:
+def is_fused(args, layers) -> bool:
+    """An NVFP4 MLP pair runs as one fused MLP block unless --unfused."""
+    return (args.config in (2, 3) and layers[0].fmt == "nvfp4_g16" and not getattr(args, "unfused", False)
+            and len(layers) == 2)
+
+
+def workload_desc(cfg: int, layers, fused: bool = False) -> str:
     L = layers[0]
+    if fused:
+        return (f"FLUX-like MLP block, fused: up [{L.M},{L.K}]x[{L.K},{L.N}] -> GELU of the up output -> down "
+                f"[{L.M},{layers[1].K}]x[{layers[1].K},{layers[1].N}], rank {L.rank}, {L.fmt}")
     if cfg == 1:
         return f"FLUX-like attention projection: X bf16 [{L.M},{L.K}] x W [{L.K},{L.N}], rank {L.rank}, {L.fmt}"
     if cfg in (2, 3):
@@ -112,23 +121,31 @@ def ws_bytes_lower_bound(L) -> int:
     return codes + scales + M_pad * ((L.rank + 31) // 32 * 32) * 2
 
 
-def rotation_sets(layers) -> tuple[int, int]:
+def rotation_sets(layers, fused: bool = False) -> tuple[int, int]:
     """(sets, bytes per set): enough rotating copies of inputs, outputs,
     workspace and prepared weights that one step's data is out of L2 again
-    when its set comes back."""
+    when its set comes back. The fused MLP block reads only the first layer's
+    X and writes only the last layer's Y."""
     set_bytes = 0
-    for L in layers:
-        set_bytes += L.M * L.K * 2 + L.M * L.N * 2 + ws_bytes_lower_bound(L)
+    for i, L in enumerate(layers):
+        if not fused or i == 0:
+            set_bytes += L.M * L.K * 2
+        if not fused or i == len(layers) - 1:
+            set_bytes += L.M * L.N * 2
+        set_bytes += ws_bytes_lower_bound(L)
         set_bytes += L.N * L.K // 2 * (2 if L.fmt == "int4_g64" else 1) + L.N * L.K // 16
     return max(2, math.ceil(2 * L2_BYTES / max(set_bytes, 1))), set_bytes
 
 
 def config_dict(args, layers) -> dict:
     """The `config` object of the JSON line, identical in both arms."""
-    n_sets, set_bytes = rotation_sets(layers)
+    fused = is_fused(args, layers)
+    n_sets, set_bytes = rotation_sets(layers, fused)
     L = layers[0]
-    return {"workload": workload_desc(args.config, layers), "config_id": args.config,
+    return {"workload": workload_desc(args.config, layers, fused), "config_id": args.config,
             "M": L.M, "K": L.K, "N": L.N, "rank": L.rank, "format": L.fmt, "layers_per_step": len(layers),
+            "pipeline": ("fused MLP block (activation kernel, up GEMM with GELU and the down layer's quantization "
+                         "in its epilogue, T sum, down GEMM)" if fused else "one forward per layer"),
             "l2": f"inputs larger than L2: {n_sets} rotating sets of prepared layer + X/Y/workspace "
                   f"(>= {n_sets * set_bytes / 2**20:.0f} MiB > 2 x 126 MiB L2)"}
 
@@ -275,15 +292,26 @@ def run_ours(args):
     peaks, peak_kind = read_peaks()
 
     # ---- prepare: one layer instance per rotating set (the first with the GPU
-    # SVD, the others from its factors), plus X / Y / workspace per set
+    # SVD, the others from its factors), plus X / Y / workspace per set. The
+    # fused MLP block's down layer is calibrated on the GELU of the up layer's
+    # output, which is what it receives.
+    fused = is_fused(args, layers)
     preps = []
-    for L in layers:
-        X0 = L.X.to(dev)
-        a = rq.calibrate_absmax(X0)
+    for li, L in enumerate(layers):
+        if fused and li == 1:
+            with torch.no_grad():
+                g_up0 = preps[0][3]
+                h = torch.nn.functional.gelu(g_up0.forward(preps[0][1]).float()).to(torch.bfloat16)
+            X0 = None
+            a = rq.calibrate_absmax(h)
+            del h
+        else:
+            X0 = L.X.to(dev)
+            a = rq.calibrate_absmax(X0)
         g0 = rq.Layer.prepare(L.W.to(dev), L.bias.to(dev), a, L.fmt, L.rank, alpha=L.alpha)
         ex = g0.export()
         preps.append((L, X0, a, g0, ex))
-    n_sets, _ = rotation_sets(layers)
+    n_sets, _ = rotation_sets(layers, fused)
     sets = []
     for s in range(n_sets):
         items = []
@@ -294,24 +322,36 @@ def run_ours(args):
                 L1 = torch.from_numpy(ex["L1"]).to(torch.bfloat16).to(dev)
                 L2 = torch.from_numpy(ex["L2"]).to(torch.bfloat16).to(dev)
                 g = rq.Layer.prepare(L.W.to(dev), L.bias.to(dev), a, L.fmt, L.rank, alpha=L.alpha, factors=(L1, L2))
-            X = X0 if s == 0 else X0.clone()
-            Y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device=dev)
-            ws = torch.empty(g.workspace_size(L.M), dtype=torch.uint8, device=dev)
-            items.append((g, X, Y, ws))
+            X = None if X0 is None else (X0 if s == 0 else X0.clone())
+            Y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device=dev) if not fused or L is layers[-1] else None
+            ws = None if fused else torch.empty(g.workspace_size(L.M), dtype=torch.uint8, device=dev)
+            items.append([g, X, Y, ws])
+        if fused:
+            blk = rq.MlpBlock(items[0][0], items[1][0])
+            items[0][3] = torch.empty(blk.workspace_size(layers[0].M), dtype=torch.uint8, device=dev)
+            items.append(blk)
         sets.append(items)
     torch.cuda.synchronize()
 
     n_layers = len(layers)
     K_steps, W_steps = args.steps, args.warmup
-    # events: per step and layer, before K1 / between / after the GEMM
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_layers)] for _ in range(K_steps)]
+    # events: per step and layer, before K1 / between / after the GEMM; the
+    # fused block records five: before K1, after K1, after the fused up GEMM,
+    # after the T sum, after the down GEMM
+    n_ev = [5] if fused else [3] * n_layers
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(n)] for n in n_ev] for _ in range(K_steps)]
     for per_step in evs:  # torch creates the CUDA event at its first record
         for per_layer in per_step:
             for e in per_layer:
                 e.record()
 
     def step(i, events=None):
-        for li, (g, X, Y, ws) in enumerate(sets[i % n_sets]):
+        items = sets[i % n_sets]
+        if fused:
+            blk = items[2]
+            blk.forward(items[0][1], out=items[1][2], workspace=items[0][3], events=None if events is None else events[0])
+            return
+        for li, (g, X, Y, ws) in enumerate(items):
             if events is None:
                 g.forward(X, out=Y, workspace=ws)
             else:
@@ -339,8 +379,15 @@ def run_ours(args):
     t1_wall = time.time()
     clocks = sampler.stop(t0_wall, t1_wall)
     elapsed_ms = start.elapsed_time(end)
-    k1_ms = [statistics.fmean(evs[i][li][0].elapsed_time(evs[i][li][1]) for i in range(K_steps)) for li in range(n_layers)]
-    gemm_ms = [statistics.fmean(evs[i][li][1].elapsed_time(evs[i][li][2]) for i in range(K_steps)) for li in range(n_layers)]
+    mean_ms = lambda li, a, b: statistics.fmean(evs[i][li][a].elapsed_time(evs[i][li][b]) for i in range(K_steps))
+    if fused:
+        k1_ms = [mean_ms(0, 0, 1)]
+        gemm_ms = [mean_ms(0, 1, 2), mean_ms(0, 3, 4)]
+        reduce_ms = mean_ms(0, 2, 3)
+    else:
+        k1_ms = [mean_ms(li, 0, 1) for li in range(n_layers)]
+        gemm_ms = [mean_ms(li, 1, 2) for li in range(n_layers)]
+        reduce_ms = None
     max_ms = max_over_ranks(elapsed_ms, world, dev)
 
     step_ops = sum(layer_ops(L.M, L.K, L.N, L.rank) for L in layers)
@@ -354,10 +401,12 @@ def run_ours(args):
     # duplex) while step i computes; events keep each rotating set's buffers
     # from being overwritten before the step that last used them is done.
     e2e_steps = max(3, min(args.e2e_steps, K_steps))
-    hostX = [L.X.pin_memory() for L in layers]
-    hostY = [torch.empty(L.M, L.N, dtype=torch.bfloat16).pin_memory() for L in layers]
-    h2d = sum(L.M * L.K * 2 for L in layers)
-    d2h = sum(L.M * L.N * 2 for L in layers)
+    io = [0] if fused else list(range(n_layers))  # layers whose X comes from the host
+    oo = [n_layers - 1] if fused else list(range(n_layers))  # layers whose Y goes back
+    hostX = {li: layers[li].X.pin_memory() for li in io}
+    hostY = {li: torch.empty(layers[li].M, layers[li].N, dtype=torch.bfloat16).pin_memory() for li in oo}
+    h2d = sum(layers[li].M * layers[li].K * 2 for li in io)
+    d2h = sum(layers[li].M * layers[li].N * 2 for li in oo)
     comp = torch.cuda.current_stream()
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
 
@@ -369,21 +418,24 @@ def run_ours(args):
             with torch.cuda.stream(s_in):
                 if fwd_done[k] is not None:
                     s_in.wait_event(fwd_done[k])
-                for li, (g, X, Y, ws) in enumerate(sets[k]):
-                    X.copy_(hostX[li], non_blocking=True)
+                for li in io:
+                    sets[k][li][1].copy_(hostX[li], non_blocking=True)
                 ev_in = torch.cuda.Event()
                 ev_in.record(s_in)
             comp.wait_event(ev_in)
             if out_done[k] is not None:
                 comp.wait_event(out_done[k])
-            for li, (g, X, Y, ws) in enumerate(sets[k]):
-                g.forward(X, out=Y, workspace=ws, stream=comp)
+            if fused:
+                sets[k][2].forward(sets[k][0][1], out=sets[k][1][2], workspace=sets[k][0][3], stream=comp)
+            else:
+                for li, (g, X, Y, ws) in enumerate(sets[k][:n_layers]):
+                    g.forward(X, out=Y, workspace=ws, stream=comp)
             fwd_done[k] = torch.cuda.Event()
             fwd_done[k].record(comp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(fwd_done[k])
-                for li, (g, X, Y, ws) in enumerate(sets[k]):
-                    hostY[li].copy_(Y, non_blocking=True)
+                for li in oo:
+                    hostY[li].copy_(sets[k][li][2], non_blocking=True)
                 out_done[k] = torch.cuda.Event()
                 out_done[k].record(s_out)
         for ev in out_done:  # the region ends when the last output is on the host
@@ -404,8 +456,8 @@ def run_ours(args):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e_value = whole_job_tops(step_ops, e2e_steps, world, e2e_ms)
     # the last step's outputs reached the host: compare them with the device copies
-    for li, (g, X, Y, ws) in enumerate(sets[(e2e_steps - 1) % n_sets]):
-        if not torch.equal(hostY[li], Y.cpu()):
+    for li in oo:
+        if not torch.equal(hostY[li], sets[(e2e_steps - 1) % n_sets][li][2].cpu()):
             raise SystemExit("e2e: the host copy of the output differs from the device result")
 
     # ---- the 4-bit weight-only (W4A16) baseline of the abstract's speedup
@@ -414,9 +466,15 @@ def run_ours(args):
     w4a16 = None
     if not args.no_w4a16:
         w4_sets = [[rq.WeightOnlyLayer(L.W.to(dev), L.bias.to(dev)) for L in layers] for _ in range(n_sets)]
+        # the same shapes: each layer's own input and output buffers (the
+        # fused block's missing ones are made here)
+        w4_io = [[(it[1] if it[1] is not None else layers[li].X.to(dev),
+                   it[2] if it[2] is not None else torch.empty(layers[li].M, layers[li].N, dtype=torch.bfloat16,
+                                                               device=dev))
+                  for li, it in enumerate(st[:n_layers])] for st in sets]
 
         def w4_step(i):
-            for li, (g, X, Y, ws) in enumerate(sets[i % n_sets]):
+            for li, (X, Y) in enumerate(w4_io[i % n_sets]):
                 w4_sets[i % n_sets][li].forward(X, out=Y)
 
         for i in range(max(3, W_steps)):
@@ -442,7 +500,7 @@ def run_ours(args):
 
     # device status: no kernel gave up a wait
     for items in sets:
-        for (g, X, Y, ws) in items:
+        for (g, X, Y, ws) in items[:n_layers]:
             if g.device_status() != rq.Status.OK:
                 raise SystemExit("a kernel reported a timed-out pipeline wait")
 
@@ -453,7 +511,7 @@ def run_ours(args):
 
     # ---- roofline of the dominant kernel (the GEMM) and of the activation kernel
     fmt = layers[0].fmt
-    wl_key = f"cfg{args.config}_M{layers[0].M}_r{layers[0].rank}_{fmt}"
+    wl_key = f"cfg{args.config}_M{layers[0].M}_r{layers[0].rank}_{fmt}" + ("_fused" if fused else "")
     g_ops = sum(gemm_ops(L.M, L.K, L.N, L.rank) for L in layers)
     g_s = sum(gemm_ms) * 1e-3
     tensor_peak, peak_desc = tensor_peak_for(peaks, fmt, elapsed_ms * 1e-3)
@@ -464,7 +522,7 @@ def run_ours(args):
                 "traffic": traffic,
                 "peak_source": f"{peak_kind} {peak_desc}",
                 "algorithmic": "2MKN + 2MrN per launch", "frac_of_datasheet_dense": g_ops / g_s / 1e12 / DATASHEET_TOPS[fmt]}
-    k_bytes = sum(k1_bytes(L.M, L.K, L.rank, fmt) for L in layers)
+    k_bytes = sum(k1_bytes(L.M, L.K, L.rank, fmt) for L in (layers[:1] if fused else layers))
     k_s = sum(k1_ms) * 1e-3
     k1_roof = {"bound": "hbm", "kernel": "act_quant_kernel", "achieved": k_bytes / k_s / 1e9, "peak": peaks["hbm_gbs"],
                "unit": "GB/s", "frac": k_bytes / k_s / 1e9 / peaks["hbm_gbs"],
@@ -492,11 +550,12 @@ def run_ours(args):
         "config": config_dict(args, layers),
         "pct_of_datasheet_dense_peak": 100.0 * value / DATASHEET_TOPS[fmt],
         "roofline": roofline,
-        "kernels": {"act_quant": {"ms": k1_ms, **k1_roof}, "gemm": {"ms": gemm_ms}},
+        "kernels": {"act_quant": {"ms": k1_ms, **k1_roof}, "gemm": {"ms": gemm_ms},
+                    **({"t_sum": {"ms": reduce_ms}} if fused else {})},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps},
-        "gpu_launches": 2 * n_layers * K_steps,
+        "gpu_launches": (4 if fused else 2 * n_layers) * K_steps,
         "w4a16_baseline": w4a16,
         "clocks": clocks,
         "impl": "ours",
@@ -665,6 +724,8 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-w4a16", action="store_true", help="skip timing the weight-only baseline")
+    ap.add_argument("--unfused", action="store_true",
+                    help="run an NVFP4 MLP pair as two layer forwards instead of the fused MLP block")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ablation", action="store_true",
                     help="print the error / time table of the method's ablations instead of the benchmark line")

@@ -169,6 +169,38 @@ SVDQ_API svdq_status svdq_linear_forward(svdq_layer_t layer, const void* X, int 
 SVDQ_API svdq_status svdq_linear_forward_profiled(svdq_layer_t layer, const void* X, int M, void* Y, void* workspace,
                                                   size_t workspace_bytes, void* stream, void* const* events);
 
+/* The MLP block of two layers, Y = down(GELU(up(X))), fused across the
+ * boundary between them: the up layer's GEMM epilogue rounds its output to
+ * bf16, applies GELU (the erf form, in float32) and rounds to bf16 (h, what a
+ * plain composition of the layers would pass on), then smooths and quantizes
+ * h for the down layer straight into the down layer's activation codes and
+ * scales, and contracts it with the down layer's factor for the down layer's
+ * branch input T. h itself never goes to device memory. Abstract: the
+ * low-rank branch is fused into the low-bit kernels to cut redundant memory
+ * traffic; this carries that across the two layers of the block.
+ * Kernels on `stream`: the up layer's activation kernel, the fused up GEMM, a
+ * small fixed-order sum of the T partials, the down layer's GEMM.
+ *   up, down  NVFP4 layers on the same device, up->N == down->K,
+ *             down->K % 256 == 0, down rank (with adapters) 1..32
+ *   X         device bf16 [M, K_up];  Y  device bf16 [M, N_down] (overwritten)
+ *   workspace at least svdq_mlp_workspace_size(up, down, M) bytes, 256-byte
+ *             aligned, no initialisation needed
+ * Other layer pairs return SVDQ_ERR_UNSUPPORTED (run them as two forwards). */
+SVDQ_API svdq_status svdq_mlp_workspace_size(svdq_layer_t up, svdq_layer_t down, int M, size_t* bytes);
+SVDQ_API svdq_status svdq_mlp_forward(svdq_layer_t up, svdq_layer_t down, const void* X, int M, void* Y,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+/* svdq_mlp_forward recording events[0..4] (cudaEvent_t) before the activation
+ * kernel, after it, after the fused up GEMM, after the T sum and after the
+ * down GEMM. */
+/* Where a forward leaves the down layer's activations in the MLP workspace
+ * (for inspection): offsets[0] codes, offsets[1] scales, offsets[2] T, in
+ * bytes from the workspace start, in the layouts svdq_quantize_activations
+ * documents for the down layer (M_pad = M rounded up to 128 rows). */
+SVDQ_API svdq_status svdq_mlp_workspace_layout(svdq_layer_t up, svdq_layer_t down, int M, size_t* offsets);
+SVDQ_API svdq_status svdq_mlp_forward_profiled(svdq_layer_t up, svdq_layer_t down, const void* X, int M, void* Y,
+                                               void* workspace, size_t workspace_bytes, void* stream,
+                                               void* const* events);
+
 /* svdq_linear_forward for callers that cannot allocate device memory: hosts
  * whose device memory belongs to their own allocator and may not be grown
  * behind its back, or latency-critical loops where an allocation may

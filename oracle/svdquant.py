@@ -311,3 +311,32 @@ def dequantize_weight_only(p: WeightOnly) -> np.ndarray:
 def forward_weight_only(p: WeightOnly, X) -> np.ndarray:
     """Y = X w^T + b in float64 with X in bf16 (the activations stay 16-bit)."""
     return np.asarray(X, dtype=np.float64) @ dequantize_weight_only(p).T + p.bias[None, :]
+
+
+# ---------------------------------------------------------------------------
+# the MLP block: up layer, GELU, down layer
+# ---------------------------------------------------------------------------
+
+def gelu_erf(x) -> np.ndarray:
+    """GELU(x) = x * Phi(x) = 0.5 x (1 + erf(x / sqrt 2)) in float64 (the exact
+    form; scipy's erf is the library step)."""
+    from scipy.special import erf
+    x = np.asarray(x, dtype=np.float64)
+    return 0.5 * x * (1.0 + erf(x / np.sqrt(2.0)))
+
+
+@dataclass
+class MlpResult:
+    y_up: np.ndarray  # float64 holding bf16 values [M, N_up]: the up layer's stored output
+    h: np.ndarray  # float64 holding bf16 values [M, N_up]: GELU(y_up), the down layer's input
+    down: ForwardResult  # the down layer's forward on h
+
+
+def mlp_forward(p_up: Prepared, p_down: Prepared, X) -> MlpResult:
+    """An MLP block of two SVDQuant layers: Y = down(GELU(up(X))). Each tensor
+    between the layers is held in bf16, as a plain composition of the layers
+    would store it: the up layer's output is rounded to bf16, GELU is applied
+    to that and rounded to bf16, and the down layer runs on the result."""
+    y_up = bf16_round(forward(p_up, X).Y)
+    h = bf16_round(gelu_erf(y_up))
+    return MlpResult(y_up, h, forward(p_down, h))

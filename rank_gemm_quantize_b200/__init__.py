@@ -88,6 +88,10 @@ SIGNATURES = {
     "svdq_last_error": [],
     "svdq_selftest_bounded_wait": [ctypes.c_ulonglong, _VP],
     "svdq_debug_fail_allocation": [ctypes.c_longlong],
+    "svdq_mlp_workspace_size": [_VP, _VP, _I, ctypes.POINTER(_SZ)],
+    "svdq_mlp_workspace_layout": [_VP, _VP, _I, ctypes.POINTER(_SZ)],
+    "svdq_mlp_forward": [_VP, _VP, _VP, _I, _VP, _VP, _SZ, _VP],
+    "svdq_mlp_forward_profiled": [_VP, _VP, _VP, _I, _VP, _VP, _SZ, _VP, ctypes.POINTER(_VP)],
     "svdq_w4a16_prepare": [_VP, _VP, _I, _I, _VP, ctypes.POINTER(_VP)],
     "svdq_w4a16_forward": [_VP, _VP, _I, _VP, _VP],
     "svdq_w4a16_export": [_VP, _VP, _VP, _VP],
@@ -399,3 +403,50 @@ class WeightOnlyLayer:
             self.close()
         except Exception:
             pass
+
+
+class MlpBlock:
+    """Y = down(GELU(up(X))) for two prepared NVFP4 layers, with GELU and the
+    down layer's quantization fused into the up layer's GEMM epilogue."""
+
+    def __init__(self, up: Layer, down: Layer):
+        self.up, self.down = up, down
+        self._ws: Optional[torch.Tensor] = None
+
+    def workspace_size(self, M: int) -> int:
+        n = ctypes.c_size_t()
+        _check(lib().svdq_mlp_workspace_size(self.up._h, self.down._h, M, ctypes.byref(n)))
+        return n.value
+
+    def workspace_layout(self, M: int):
+        """(codes, scales, T) byte offsets of the down layer's activations in the workspace."""
+        off = (ctypes.c_size_t * 3)()
+        _check(lib().svdq_mlp_workspace_layout(self.up._h, self.down._h, M, off))
+        return tuple(off)
+
+    def workspace(self, M: int) -> torch.Tensor:
+        need = self.workspace_size(M)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=self.up.device)
+        return self._ws
+
+    def forward(self, X: torch.Tensor, out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                stream=None, events=None) -> torch.Tensor:
+        self.up._check_io(X, None, workspace)
+        M = X.shape[0]
+        N = self.down.info().N
+        if out is None:
+            out = torch.empty(M, N, dtype=torch.bfloat16, device=X.device)
+        elif tuple(out.shape) != (M, N) or out.dtype != torch.bfloat16 or not out.is_contiguous():
+            raise ValueError(f"out must be a contiguous bfloat16 [{M}, {N}] tensor")
+        ws = workspace if workspace is not None else self.workspace(M)
+        if events is None:
+            _check(lib().svdq_mlp_forward(self.up._h, self.down._h, _ptr(X), M, _ptr(out), _ptr(ws), ws.numel(),
+                                          _stream(stream)))
+        else:
+            arr = (ctypes.c_void_p * 5)(*[e.cuda_event for e in events])
+            _check(lib().svdq_mlp_forward_profiled(self.up._h, self.down._h, _ptr(X), M, _ptr(out), _ptr(ws),
+                                                   ws.numel(), _stream(stream), arr))
+        return out
+
+    __call__ = forward

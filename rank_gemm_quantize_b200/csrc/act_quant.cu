@@ -90,13 +90,13 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 // k0 .. k0+15) and store their codes and group scale.
 template <int FMT>
 __device__ __forceinline__ void quantize16(const float (&v)[16], const ActQuantParams& p, int row, int k0, int seg) {
-  float m[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) m[i] = fmaxf(fabsf(v[2 * i]), fabsf(v[2 * i + 1]));
-#pragma unroll
-  for (int i = 0; i < 4; ++i) m[i] = fmaxf(m[i], m[i + 4]);
-  float amax = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
   if (FMT == SVDQ_INT4_G64) {
+    float m[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = fmaxf(fabsf(v[2 * i]), fabsf(v[2 * i + 1]));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m[i] = fmaxf(m[i], m[i + 4]);
+    float amax = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
     // a group of 64 = the 4 lanes of this row (lane >> 2 shared)
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
@@ -120,20 +120,8 @@ __device__ __forceinline__ void quantize16(const float (&v)[16], const ActQuantP
     if (seg == 0) reinterpret_cast<float*>(p.scales)[static_cast<size_t>(k0 >> 6) * p.M_pad + row] = scale;
   } else {
     // a group of 16 = this thread's values
-    const uint32_t sb = cvt_e4m3x2(__fdiv_rn(amax, p.denom), 0.f) & 0xFFu;
-    const float eff = __fmul_rn(e4m3_to_float(sb), p.g_x);
-    const float inv = __frcp_rn(eff != 0.f ? eff : 1.f);
-    float q[2][8];
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-      for (int j = 0; j < 8; j += 2) {
-        const float2 pr = __fmul2_rn(make_float2(v[8 * h + j], v[8 * h + j + 1]), make_float2(inv, inv));
-        q[h][j] = pr.x;
-        q[h][j + 1] = pr.y;
-      }
-    const uint32_t c0 = eff != 0.f ? cvt_e2m1x8(q[0]) : 0u;
-    const uint32_t c1 = eff != 0.f ? cvt_e2m1x8(q[1]) : 0u;
+    uint32_t c0, c1;
+    const uint32_t sb = nvfp4_quant16(v, p.denom, p.g_x, c0, c1);
     *reinterpret_cast<uint2*>(p.codes + static_cast<size_t>(row) * (p.K >> 1) + (k0 >> 1)) = make_uint2(c0, c1);
     // scale-factor atom: (row / 128) * (K / 64) + k / 64, byte (row % 32) * 16 + ((row / 32) % 4) * 4 + (k / 16) % 4
     const size_t atom = static_cast<size_t>(row >> 7) * (p.K >> 6) + (k0 >> 6);

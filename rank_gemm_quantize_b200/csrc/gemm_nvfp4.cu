@@ -12,26 +12,44 @@
 // low-rank term never makes a separate pass over Y; the epilogue applies the
 // tensor scales and the bias and stores bf16 once.
 //
-// Persistent kernel, one CTA per SM, 128 x 256 output tiles taken round-robin.
-// Warp roles (11 warps):
-//   warp 0  producer: for each tile, a bulk copy of the bias slice, then the
-//           k-tiles (A and B codes by TMA, their scale-factor atoms by bulk
-//           copy) followed by the branch k-tiles (a 32-column slice of T'
-//           and of L2^T), through a 4-stage shared-memory ring;
-//   warp 10 scale factors: copies each stage's scale-factor atoms into that
-//           stage's TMEM slot with tcgen05.cp and commits them to the stage's
-//           sf_ready barrier. Copies issued from the MMA thread serialise
-//           with its MMAs (about 47 cycles per copy, 12 per k-tile, against
-//           512 cycles of MMAs); from a thread of their own they overlap;
-//   warp 1  TMEM owner and MMA issuer (one thread): per k-tile, once the
-//           stage's scale factors are in TMEM, 4 block-scaled MMAs; per
-//           branch k-tile 2 kind::f16 MMAs; commits release the stage / mark
-//           the tile;
-//   warps 2-9 epilogue: each copies its 32 rows x 128 columns of the
-//           accumulator to registers and releases TMEM at once, so the next
-//           tile's MMAs overlap the scaling, bias and bf16 stores.
-// Tiles are ordered with the N index fastest so the CTAs in flight share the
-// weight panel in L2.
+// Two SMs work as one (a cluster of two CTAs, tcgen05 .cta_group::2): the
+// pair computes a 256 x 256 output tile with M = 256 MMAs. Each CTA loads
+// only its own 128 rows of the activation codes and its own 128 columns of the
+// weight codes (plain TMA, no multicast), plus its rows' activation scale
+// factors and the weight scale factors of all 256 columns; the tensor cores
+// of the pair read both CTAs' halves. Per SM that is 38 KB of operands per
+// 256-deep k-tile instead of 54 KB for a 128 x 256 tile on one SM.
+//
+// Persistent kernel, one pair per two SMs. Warp roles (11 warps per CTA):
+//   warp 0  producer (both CTAs): per tile its bias slice (bulk copy, local
+//           ring), then the k-tiles: A and B codes and both scale-factor
+//           tiles by TMA, completing on the leader CTA's stage barrier;
+//           then the branch k-tiles (32-column slices of T' and L2^T);
+//   warp 10 scale factors (leader): copies each stage's scale factors of both
+//           CTAs into their TMEM (tcgen05.cp .cta_group::2) and commits;
+//   warp 1  TMEM owner (both) and MMA issuer (leader, one thread): per k-tile
+//           4 block-scaled MMAs, per branch k-tile 2 kind::f16 MMAs; the
+//           commits free the stage in both CTAs and mark the tile;
+//   warps 2-9 epilogue (both): each reads its 32 rows x 128 columns of its
+//           CTA's accumulator 32 columns at a time, scales, adds the bias,
+//           packs bf16 and writes it into a 128-byte-swizzled staging buffer
+//           right away; then it tells the leader that TMEM is free (the next
+//           tile's MMAs start) and stores its two 32 x 64 boxes with TMA
+//           (rows and columns past M and N are clipped by the tensor map).
+//
+// MLP-block variant (kMlp, the up layer of up -> GELU -> down): the epilogue
+// does not store Y. It rounds the output to bf16, applies GELU (erf form,
+// float32) and rounds to bf16 (h: the tensor a plain composition of the two
+// layers would pass on), then smooths and NVFP4-quantizes h for the down
+// layer into that layer's code and scale buffers, and stages h in shared
+// memory. The leader then contracts the staged h with the down layer's
+// 1/s-folded factor (L1s^T slices loaded per tile) into a TMEM accumulator:
+// the down layer's branch input T. A pair takes a contiguous range of tiles
+// in row-major tile order, so T accumulates over the pair's tiles of one
+// 256-row block; it is flushed as a float partial when the row block changes
+// and the partials are summed in a fixed order by nvfp4_mlp_t_reduce. The
+// contraction of tile i is issued after the next tile's mainloop MMAs, so it
+// overlaps the epilogue instead of waiting for it.
 #include <cstdint>
 
 #include "common.cuh"
@@ -41,204 +59,341 @@ namespace svdq {
 
 namespace {
 
-constexpr int kBM = 128;
-constexpr int kBN = 256;
+constexpr int kBM = 128;       // rows per CTA (the pair covers 256)
+constexpr int kBN = 256;       // columns per pair tile
+constexpr int kBNHalf = 128;   // weight rows each CTA loads
 constexpr int kBKBytes = 128;  // 256 E2M1 values per row per k-tile
-constexpr int kStages = 4;
 constexpr int kEpiWarps = 8;
 constexpr int kCpWarp = 2 + kEpiWarps;  // copies scale factors into TMEM
 constexpr int kThreads = (3 + kEpiWarps) * 32;
 
+template <bool kMlp>
 struct SmemNv {
-  static constexpr int kA = kBM * kBKBytes;   // 16 KB
-  static constexpr int kB = kBN * kBKBytes;   // 32 KB
-  static constexpr int kSfa = 4 * 512;        // 4 k-blocks of 64
-  static constexpr int kSfb = (kBN / 128) * 4 * 512;
-  static constexpr int kStage = kA + kB + kSfa + kSfb;
+  static constexpr int kStages = kMlp ? 3 : 4;
+  static constexpr int kA = kBM * kBKBytes;       // 16 KB
+  static constexpr int kB = kBNHalf * kBKBytes;   // 16 KB
+  static constexpr int kSfa = 4 * 512;            // this CTA's 128 rows, 4 k-blocks of 64
+  static constexpr int kSfb = (kBN / 128) * 4 * 512;  // all 256 columns, 4 k-blocks
+  static constexpr int kStage = kA + kB + kSfa + kSfb;  // 38 KB
   static constexpr int kBiasOff = kStages * kStage;
-  static constexpr int kBias = kBN * 2;       // bf16 bias slice of a tile
-  static constexpr int kBarOff = kBiasOff + 2 * kBias;
-  static constexpr int kTotal = kBarOff + 256 + 1024;
+  static constexpr int kBias = kBN * 2;           // bf16 bias slice of a tile
+  // Y staging for the TMA stores (8 warps x two 32 x 64 boxes); in the MLP
+  // variant the same 64 KB hold h as four K-major 128 x 64 bf16 chunks.
+  static constexpr int kStgOff = kBiasOff + 2 * kBias;
+  static constexpr int kStgBox = 32 * 128;
+  static constexpr int kStgWarp = 2 * kStgBox;
+  static constexpr int kStg = kEpiWarps * kStgWarp;  // 64 KB
+  static constexpr int kHChunk = kBM * 128;          // 16 KB: 128 rows x 64 bf16
+  static constexpr int kIsOff = kStgOff + kStg;      // MLP: down-layer inv_s slices, 2 x 256 floats
+  static constexpr int kIs = kMlp ? kBN * 4 : 0;
+  static constexpr int kL1Off = kIsOff + 2 * kIs;    // MLP: down-layer L1s^T slices, 2 slots
+  static constexpr int kL1Part = (kMlpDownRP / 2) * 128;  // this CTA's 16 rows x 64 bf16 (hi or lo)
+  static constexpr int kL1Slot = kMlp ? 4 * 2 * kL1Part : 0;  // 4 chunks x (hi, lo)
+  static constexpr int kBarOff = kL1Off + 2 * kL1Slot;
+  static constexpr int kTotal = kBarOff + 512 + 1024;
 };
-static_assert(SmemNv::kTotal <= 232448, "shared memory budget");
-static_assert(kBN % kWeightBoxRows == 0 && kBM % kActBoxRows == 0, "operand tiles are whole boxes");
+static_assert(SmemNv<false>::kTotal <= 232448 && SmemNv<true>::kTotal <= 232448, "shared memory budget");
+static_assert(SmemNv<false>::kStage % 1024 == 0 && SmemNv<true>::kStgOff % 1024 == 0 &&
+                  SmemNv<false>::kStgOff % 1024 == 0 && SmemNv<true>::kL1Off % 1024 == 0,
+              "swizzled tiles start 1 KB-aligned");
+static_assert(kBNHalf == kWeightBoxRows && kBM == kActBoxRows, "each CTA loads one box per operand");
 
-// TMEM columns: accumulator [0, 256), then one scale-factor slot per
+// TMEM columns (each CTA): accumulator [0, 256), then one scale-factor slot per
 // shared-memory stage (A: 16 columns, B: 32), so copying the next k-tile's
-// scale factors never waits for the MMAs still reading the previous ones.
+// scale factors never waits for the MMAs still reading the previous ones;
+// then (MLP) the down layer's T accumulator.
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfSlotCols = 16 + 2 * 16;
 constexpr uint32_t kSfaCol = kBN;
 constexpr uint32_t kSfbCol = kBN + 16;
-static_assert(kBN + kStages * kSfSlotCols <= kTmemCols, "TMEM budget");
+template <bool kMlp>
+constexpr uint32_t t_acc_col() { return kBN + SmemNv<kMlp>::kStages * kSfSlotCols; }
+static_assert(t_acc_col<true>() + kMlpDownRP <= kTmemCols && t_acc_col<false>() <= kTmemCols, "TMEM budget");
 
-__global__ void __launch_bounds__(kThreads, 1)
-    gemm_nvfp4_kernel(const GemmParams p, const __grid_constant__ GemmMaps maps) {
-  using L = SmemNv;
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// The tile range of pair `pair`: round-robin for the plain GEMM (the pairs in
+// flight share the weight panel in L2); contiguous in row-major tile order for
+// the MLP variant (the down layer's T accumulates over a row block).
+struct TileRange {
+  int first, last, step;
+};
+template <bool kMlp>
+__device__ __forceinline__ TileRange tile_range(int pair, int n_pairs, int n_tiles) {
+  if (kMlp) {
+    return {static_cast<int>((static_cast<long long>(pair) * n_tiles) / n_pairs),
+            static_cast<int>((static_cast<long long>(pair + 1) * n_tiles) / n_pairs), 1};
+  }
+  return {pair, n_tiles, n_pairs};
+}
+
+// The first pair whose contiguous range holds a tile of 256-row block mp.
+__host__ __device__ inline int mlp_first_pair(int mp, int n_blocks, int n_tiles, int n_pairs) {
+  const long long t = static_cast<long long>(mp) * n_blocks;
+  int p = 0;
+  while (p < n_pairs - 1 && (static_cast<long long>(p + 1) * n_tiles) / n_pairs <= t) ++p;
+  return p;
+}
+
+template <bool kMlp>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    gemm_nvfp4_kernel(const GemmParams p, const MlpDownParams mlp, const __grid_constant__ GemmMaps maps) {
+  using L = SmemNv<kMlp>;
+  constexpr int kStages = L::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-  uint64_t* empty = full + kStages;
-  uint64_t* acc_full = empty + kStages;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* bias_full = acc_empty + 1;   // [2]
-  uint64_t* bias_empty = bias_full + 2;  // [2]
-  uint64_t* drain = bias_empty + 2;
-  uint64_t* sf_ready = drain + 1;        // [kStages] scale factors of the stage are in TMEM
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);  // [kStages] (leader) both CTAs' loads landed
+  uint64_t* empty = full + kStages;      // [kStages] (both) the MMAs are done with the stage
+  uint64_t* acc_full = empty + kStages;  // (both) the tile's accumulator is complete
+  uint64_t* acc_empty = acc_full + 1;    // (leader) both CTAs' epilogues copied the accumulator out
+  uint64_t* bias_full = acc_empty + 1;   // [2] (both, local)
+  uint64_t* bias_empty = bias_full + 2;  // [2] (both, local)
+  uint64_t* drain = bias_empty + 2;      // (both) every MMA has completed
+  uint64_t* sf_ready = drain + 1;        // [kStages] (leader) scale factors of the stage are in TMEM
   uint64_t* cp_done = sf_ready + kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cp_done + 1);
+  // MLP block only:
+  uint64_t* is_full = cp_done + 1;       // [2] (both, local) down-layer inv_s slice landed
+  uint64_t* is_empty = is_full + 2;      // [2] (both, local)
+  uint64_t* l1_full = is_empty + 2;      // [2] (leader) both CTAs' L1s^T slices landed
+  uint64_t* l1_empty = l1_full + 2;      // [2] (both) the T MMAs of the slot's tile completed
+  uint64_t* h_ready = l1_empty + 2;      // (leader) both CTAs staged the tile's h
+  uint64_t* t_full = h_ready + 1;        // (both) T accumulator holds a finished row-block partial
+  uint64_t* t_empty = t_full + 1;        // (leader) both CTAs read that partial out
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(t_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n_blocks = (p.N + kBN - 1) / kBN;
-  const int n_tiles = (p.M_pad / kBM) * n_blocks;
+  const uint32_t rank = cluster_ctarank();  // 0: leader (issues the MMAs), 1: peer
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+  const int n_blocks = p.N_pad / kBN;
+  const int m_pairs = (p.M_pad + 2 * kBM - 1) / (2 * kBM);
+  const int n_tiles = m_pairs * n_blocks;
   const int kb_total = p.K / 64;
   const int n_main = (p.K + 255) / 256;
   const int n_lr = p.RP / 32;
   const int n_items = n_main + n_lr;
+  const TileRange tr = tile_range<kMlp>(pair, n_pairs, n_tiles);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sf_ready[s], 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, kEpiWarps);
+    mbar_init(acc_empty, 2 * kEpiWarps);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bias_full[b], 1);
       mbar_init(&bias_empty[b], kEpiWarps);
+      mbar_init(&is_full[b], 1);
+      mbar_init(&is_empty[b], kEpiWarps);
+      mbar_init(&l1_full[b], 1);
+      mbar_init(&l1_empty[b], 1);
     }
     mbar_init(drain, 1);
-    for (int s = 0; s < kStages; ++s) mbar_init(&sf_ready[s], 1);
     mbar_init(cp_done, 1);
+    mbar_init(h_ready, 2 * kEpiWarps);
+    mbar_init(t_full, 1);
+    mbar_init(t_empty, 2 * 4);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ producer (both CTAs)
     if (lane == 0) {
       prefetch_tensormap(&maps.a);
       prefetch_tensormap(&maps.b);
+      prefetch_tensormap(&maps.sfa);
+      prefetch_tensormap(&maps.sfb);
       if (n_lr > 0) {  // no branch (rank 0): its maps are never read
         prefetch_tensormap(&maps.t);
         prefetch_tensormap(&maps.l2);
       }
+      if (kMlp) {
+        prefetch_tensormap(&maps.l1h_down);
+        prefetch_tensormap(&maps.l1l_down);
+      }
       bool ok = true;
       int it = 0;          // k-tiles issued over all tiles of this CTA
       int ti = 0;          // tiles of this CTA
-      int last_bias = -1;  // last tile whose bias copy was issued
-      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++ti) {
-        const int mb = tile / n_blocks, nb = tile % n_blocks;
-        const int m0 = mb * kBM, n0 = nb * kBN;
+      int last_bias = -1;  // last tile whose local copies were issued
+      for (int tile = tr.first; tile < tr.last && ok; tile += tr.step, ++ti) {
+        const int mp = tile / n_blocks, nb = tile % n_blocks;
+        const int m0 = mp * 2 * kBM + static_cast<int>(rank) * kBM;  // this CTA's rows
+        const int n0 = nb * kBN;
         const int bs = ti & 1;
         ok = mbar_wait(&bias_empty[bs], ((ti >> 1) & 1) ^ 1, abort_flag, p.status);
+        if (ok && kMlp) ok = mbar_wait(&is_empty[bs], ((ti >> 1) & 1) ^ 1, abort_flag, p.status);
         if (!ok) break;
         mbar_arrive_expect_tx(&bias_full[bs], L::kBias);
         bulk_load(smem + L::kBiasOff + bs * L::kBias, p.bias + n0, L::kBias, &bias_full[bs]);
+        if (kMlp) {
+          mbar_arrive_expect_tx(&is_full[bs], L::kIs);
+          bulk_load(smem + L::kIsOff + bs * L::kIs, mlp.inv_s + n0, L::kIs, &is_full[bs]);
+        }
         last_bias = ti;
         for (int k = 0; k < n_items && ok; ++k, ++it) {
           const int s = it % kStages;
           ok = mbar_wait(&empty[s], ((it / kStages) & 1) ^ 1, abort_flag, p.status);
           if (!ok) break;
           uint8_t* st = smem + s * L::kStage;
+          const uint32_t fb = leader_addr(&full[s]);
           if (k < n_main) {
+            if (leader) mbar_arrive_expect_tx(&full[s], 2 * L::kStage);
             const int kb0 = k * 4;
-            const int nkb = min(4, kb_total - kb0);
-            mbar_arrive_expect_tx(&full[s], L::kA + L::kB + nkb * 512 * (1 + kBN / 128));
+            tma_load_2d_pair(st, &maps.a, fb, k * kBKBytes, m0);
+            tma_load_2d_pair(st + L::kA, &maps.b, fb, k * kBKBytes, n0 + static_cast<int>(rank) * kBNHalf);
+            // scale-factor atoms (512 bytes each): 4 k-blocks of this CTA's row block, and of both column blocks
+            tma_load_2d_pair(st + L::kA + L::kB, &maps.sfa, fb, 0, (m0 / 128) * kb_total + kb0);
 #pragma unroll
-            for (int h = 0; h < kBM / kActBoxRows; ++h)
-              tma_load_2d(st + h * kActBoxRows * kBKBytes, &maps.a, &full[s], k * kBKBytes, m0 + h * kActBoxRows);
-#pragma unroll
-            for (int h = 0; h < kBN / kWeightBoxRows; ++h)
-              tma_load_2d(st + L::kA + h * kWeightBoxRows * kBKBytes, &maps.b, &full[s], k * kBKBytes, n0 + h * kWeightBoxRows);
-            const uint8_t* sa = reinterpret_cast<const uint8_t*>(p.sa) + (static_cast<size_t>(mb) * kb_total + kb0) * 512;
-            bulk_load(st + L::kA + L::kB, sa, nkb * 512, &full[s]);
-#pragma unroll
-            for (int h = 0; h < kBN / 128; ++h) {
-              const uint8_t* sb = reinterpret_cast<const uint8_t*>(p.sb) +
-                                  (static_cast<size_t>(nb * (kBN / 128) + h) * kb_total + kb0) * 512;
-              bulk_load(st + L::kA + L::kB + L::kSfa + h * 2048, sb, nkb * 512, &full[s]);
-            }
+            for (int h = 0; h < kBN / 128; ++h)
+              tma_load_2d_pair(st + L::kA + L::kB + L::kSfa + h * 2048, &maps.sfb, fb, 0,
+                               (nb * (kBN / 128) + h) * kb_total + kb0);
           } else {
+            if (leader) mbar_arrive_expect_tx(&full[s], 2 * (kBM * 64 + kBNHalf * 64));
             const int c = k - n_main;  // 32-column slice of the branch
-            mbar_arrive_expect_tx(&full[s], kBM * 64 + kBN * 64);
-            tma_load_2d(st, &maps.t, &full[s], c * 32, m0);
+            tma_load_2d_pair(st, &maps.t, fb, c * 32, m0);
+            tma_load_2d_pair(st + L::kA, &maps.l2, fb, c * 32, n0 + static_cast<int>(rank) * kBNHalf);
+          }
+        }
+        if (kMlp && ok) {
+          // this CTA's half of the down layer's factor rows for the tile's four 64-wide K chunks. It is
+          // used by the tile's T contraction, which comes after the next tile's mainloop, so it is
+          // loaded after this tile's k-tiles: waiting for the slot (freed by the contraction of the
+          // tile two back) never delays a k-tile.
+          ok = mbar_wait(&l1_empty[bs], ((ti >> 1) & 1) ^ 1, abort_flag, p.status);
+          if (!ok) break;
+          const uint32_t lb = leader_addr(&l1_full[bs]);
+          if (leader) mbar_arrive_expect_tx(&l1_full[bs], 2 * L::kL1Slot);
+          uint8_t* l1 = smem + L::kL1Off + bs * L::kL1Slot;
 #pragma unroll
-            for (int h = 0; h < kBN / kWeightBoxRows; ++h)
-              tma_load_2d(st + L::kA + h * kWeightBoxRows * 64, &maps.l2, &full[s], c * 32,
-                          n0 + h * kWeightBoxRows);
+          for (int c = 0; c < 4; ++c) {
+            const int y = static_cast<int>(rank) * (kMlpDownRP / 2);
+            tma_load_2d_pair(l1 + (2 * c) * L::kL1Part, &maps.l1h_down, lb, n0 + 64 * c, y);
+            tma_load_2d_pair(l1 + (2 * c + 1) * L::kL1Part, &maps.l1l_down, lb, n0 + 64 * c, y);
           }
         }
       }
       if (!ok) {
-        // gave up: let the copies already in flight land before the CTA exits
+        // gave up: let this CTA's local copies in flight land before it exits
         volatile int no_abort = 0;
-        for (int j = max(0, it - kStages); j < it; ++j) mbar_wait(&full[j % kStages], (j / kStages) & 1, &no_abort, nullptr);
         for (int t2 = last_bias - 1; t2 <= last_bias; ++t2)
-          if (t2 >= 0) mbar_wait(&bias_full[t2 & 1], (t2 >> 1) & 1, &no_abort, nullptr);
+          if (t2 >= 0) {
+            mbar_wait(&bias_full[t2 & 1], (t2 >> 1) & 1, &no_abort, nullptr);
+            if (kMlp) mbar_wait(&is_full[t2 & 1], (t2 >> 1) & 1, &no_abort, nullptr);
+          }
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    const uint32_t idesc_main = idesc_block_scaled(kBM, kBN);
-    const uint32_t idesc_lr = idesc_dense(kFmtF32, kFmtBF16, kFmtBF16, kBM, kBN);
-    bool ok = true;
-    int it = 0, ti = 0;
-    for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++ti) {
-      // the epilogue has copied the previous tile's accumulator out of TMEM
-      ok = mbar_wait(acc_empty, (ti & 1) ^ 1, abort_flag, p.status);
-      if (!ok) break;
-      tc_fence_after();
-      for (int k = 0; k < n_items && ok; ++k, ++it) {
-        const int s = it % kStages;
-        ok = mbar_wait(&sf_ready[s], (it / kStages) & 1, abort_flag, p.status);
-        if (!ok) break;
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (leader) {
+      const uint32_t idesc_main = idesc_block_scaled(2 * kBM, kBN);
+      const uint32_t idesc_lr = idesc_dense(kFmtF32, kFmtBF16, kFmtBF16, 2 * kBM, kBN);
+      const uint32_t idesc_t = idesc_dense(kFmtF32, kFmtBF16, kFmtBF16, 2 * kBM, kMlpDownRP);
+      bool ok = true;
+      int it = 0, ti = 0;
+      int flushes = 0;  // MLP: row-block partials of T flushed so far
+      // MLP: the down layer's T contraction of tile j (issued after tile j+1's mainloop)
+      auto issue_t = [&](int j, int tile_j) -> bool {
+        const int mp = tile_j / n_blocks;
+        const bool first = tile_j == tr.first || (tile_j - 1) / n_blocks != mp;
+        const bool last = tile_j + 1 == tr.last || (tile_j + 1) / n_blocks != mp;
+        if (first && flushes > 0 && !mbar_wait(t_empty, (flushes - 1) & 1, abort_flag, p.status)) return false;
+        if (!mbar_wait(&l1_full[j & 1], (j >> 1) & 1, abort_flag, p.status)) return false;
+        if (!mbar_wait(h_ready, j & 1, abort_flag, p.status)) return false;
         tc_fence_after();
-        if (lane == 0) {  // one fixed thread issues every tcgen05 op, so its commits track them all
-          uint8_t* st = smem + s * L::kStage;
-          const uint32_t a_base = smem_u32(st);
-          const uint32_t b_base = smem_u32(st + L::kA);
-          if (k < n_main) {
-            const int nkb = min(4, kb_total - k * 4);
-            const uint32_t t_sfa = tmem + kSfaCol + s * kSfSlotCols;
-            const uint32_t t_sfb = tmem + kSfbCol + s * kSfSlotCols;
-            for (int j = 0; j < nkb; ++j) {
-              const uint64_t ad = smem_desc(a_base + 32 * j, 16, 1024, kSw128);
-              const uint64_t bd = smem_desc(b_base + 32 * j, 16, 1024, kSw128);
-              mma_nvf4(tmem, ad, bd, idesc_main, t_sfa + 4 * j, t_sfb + (kBN / 32) * j, (k > 0 || j > 0) ? 1u : 0u);
-            }
-          } else {
+        if (lane == 0) {
+          const uint32_t hst = smem_u32(smem + L::kStgOff);
+          const uint32_t l1 = smem_u32(smem + L::kL1Off + (j & 1) * L::kL1Slot);
+          const uint32_t tacc = tmem + t_acc_col<kMlp>();
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const uint64_t ad = smem_desc(a_base + 32 * j, 16, 512, kSw64);
-              const uint64_t bd = smem_desc(b_base + 32 * j, 16, 512, kSw64);
-              mma_f16(tmem, ad, bd, idesc_lr, 1u);
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t ad = smem_desc(hst + c * L::kHChunk + 32 * ks, 16, 1024, kSw128);
+              mma_f16_pair(tacc, ad, smem_desc(l1 + (2 * c) * L::kL1Part + 32 * ks, 16, 1024, kSw128), idesc_t,
+                           (first && c == 0 && ks == 0) ? 0u : 1u);
+              mma_f16_pair(tacc, ad, smem_desc(l1 + (2 * c + 1) * L::kL1Part + 32 * ks, 16, 1024, kSw128), idesc_t,
+                           1u);
             }
-          }
-          tc_commit(&empty[s]);
-          if (k == n_items - 1) tc_commit(acc_full);
+          tc_commit_pair_mc(&l1_empty[j & 1], 0x3);
+          if (last) tc_commit_pair_mc(t_full, 0x3);
         }
         __syncwarp();
+        if (last) ++flushes;
+        return true;
+      };
+      int prev_tile = -1;
+      for (int tile = tr.first; tile < tr.last && ok; tile += tr.step, ++ti) {
+        // both CTAs' epilogues have copied the previous tile's accumulator out of TMEM
+        ok = mbar_wait(acc_empty, (ti & 1) ^ 1, abort_flag, p.status);
+        if (!ok) break;
+        tc_fence_after();
+        for (int k = 0; k < n_items && ok; ++k, ++it) {
+          const int s = it % kStages;
+          ok = mbar_wait(&sf_ready[s], (it / kStages) & 1, abort_flag, p.status);
+          if (!ok) break;
+          tc_fence_after();
+          if (lane == 0) {  // one fixed thread issues every tcgen05 op, so its commits track them all
+            uint8_t* st = smem + s * L::kStage;
+            const uint32_t a_base = smem_u32(st);
+            const uint32_t b_base = smem_u32(st + L::kA);
+            if (k < n_main) {
+              const int nkb = min(4, kb_total - k * 4);
+              const uint32_t t_sfa = tmem + kSfaCol + s * kSfSlotCols;
+              const uint32_t t_sfb = tmem + kSfbCol + s * kSfSlotCols;
+              for (int j = 0; j < nkb; ++j) {
+                const uint64_t ad = smem_desc(a_base + 32 * j, 16, 1024, kSw128);
+                const uint64_t bd = smem_desc(b_base + 32 * j, 16, 1024, kSw128);
+                mma_nvf4_pair(tmem, ad, bd, idesc_main, t_sfa + 4 * j, t_sfb + (kBN / 32) * j,
+                              (k > 0 || j > 0) ? 1u : 0u);
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 2; ++j) {
+                const uint64_t ad = smem_desc(a_base + 32 * j, 16, 512, kSw64);
+                const uint64_t bd = smem_desc(b_base + 32 * j, 16, 512, kSw64);
+                mma_f16_pair(tmem, ad, bd, idesc_lr, 1u);
+              }
+            }
+            tc_commit_pair_mc(&empty[s], 0x3);  // the stage is free in both CTAs
+          }
+          __syncwarp();
+        }
+        if (!ok) break;
+        if (kMlp && ti > 0) {
+          ok = issue_t(ti - 1, prev_tile);
+          if (!ok) break;
+        }
+        if (lane == 0) tc_commit_pair_mc(acc_full, 0x3);  // also implies the T contraction above completed
+        __syncwarp();
+        prev_tile = tile;
       }
+      if (kMlp && ok && ti > 0) issue_t(ti - 1, prev_tile);
     }
   } else if (warp == kCpWarp) {
-    // ------------------------------------------------------------ scale factors to TMEM
+    // ------------------------------------------------------------ scale factors to TMEM (leader)
     // One stage ahead of the MMA thread at most (it waits for each stage's
     // copies): the copies and the MMAs come from different threads.
-    if (lane == 0) {
+    if (leader && lane == 0) {
       bool ok = true;
       int it = 0;
-      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+      for (int tile = tr.first; tile < tr.last && ok; tile += tr.step) {
         for (int k = 0; k < n_items && ok; ++k, ++it) {
           const int s = it % kStages;
           ok = mbar_wait(&full[s], (it / kStages) & 1, abort_flag, p.status);
@@ -252,105 +407,306 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t sfa_base = smem_u32(st + L::kA + L::kB);
             const uint32_t sfb_base = sfa_base + L::kSfa;
             for (int j = 0; j < nkb; ++j) {
-              tmem_cp_32x128b_x4(t_sfa + 4 * j, smem_desc(sfa_base + 512 * j, 16, 128, kSwNone));
+              tmem_cp_32x128b_x4_pair(t_sfa + 4 * j, smem_desc(sfa_base + 512 * j, 16, 128, kSwNone));
 #pragma unroll
               for (int h = 0; h < kBN / 128; ++h)
-                tmem_cp_32x128b_x4(t_sfb + (kBN / 32) * j + 4 * h,
-                                   smem_desc(sfb_base + h * 2048 + 512 * j, 16, 128, kSwNone));
+                tmem_cp_32x128b_x4_pair(t_sfb + (kBN / 32) * j + 4 * h,
+                                        smem_desc(sfb_base + h * 2048 + 512 * j, 16, 128, kSwNone));
             }
           }
-          tc_commit(&sf_ready[s]);
+          tc_commit_pair(smem_u32(&sf_ready[s]));
         }
       }
-      tc_commit(cp_done);  // arrives once every copy issued above has finished
+      tc_commit_pair(smem_u32(cp_done));  // arrives once every copy issued above has finished
       volatile int no_abort = 0;
       mbar_wait(cp_done, 0, &no_abort, nullptr);
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ epilogue (both CTAs)
     const int ew = warp - 2;                  // 0..7
     const int q = warp & 3;                   // TMEM lane quarter this warp may access
     const int col0 = (ew >> 2) * (kBN / 2);   // this warp's half of the tile's columns
+    const int rc = 32 * q + lane;             // this thread's row within the CTA's 128
+    uint8_t* stg = smem + L::kStgOff + ew * L::kStgWarp;
     bool ok = true;
     int ti = 0;
-    for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++ti) {
-      const int mb = tile / n_blocks, nb = tile % n_blocks;
-      const int row = mb * kBM + 32 * q + lane;
-      const int nbase = nb * kBN + col0;
-      ok = mbar_wait(acc_full, ti & 1, abort_flag, p.status);
-      if (!ok) break;
+    int flushes = 0;
+    // MLP: the pair's T partial of the row block that ended with tile_j -> workspace
+    auto flush_t = [&](int tile_j) -> bool {
+      if (!mbar_wait(t_full, flushes & 1, abort_flag, p.status)) return false;
+      ++flushes;
+      if (ew >= 4) return true;  // one warp per TMEM lane quarter reads the partial
       tc_fence_after();
-      uint32_t r[kBN / 2];
-      const uint32_t ta = tmem + (static_cast<uint32_t>(32 * q) << 16) + col0;
-#pragma unroll
-      for (int c = 0; c < kBN / 64; ++c) tmem_ld32(ta + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+      const int mp = tile_j / n_blocks;
+      const int slot = pair - mlp_first_pair(mp, n_blocks, n_tiles, n_pairs);
+      uint32_t r[32];
+      tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + t_acc_col<kMlp>(), r);
       tmem_ld_wait();
+      float* dst = mlp.tpart + ((static_cast<size_t>(mp) * mlp.slots + slot) * (2 * kBM) +
+                                static_cast<int>(rank) * kBM + rc) * kMlpDownRP;
+#pragma unroll
+      for (int e = 0; e < kMlpDownRP; e += 4)
+        *reinterpret_cast<float4*>(dst + e) = make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
+                                                          __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);  // TMEM free for the next tile's MMAs
+      if (lane == 0) mbar_arrive_cluster(t_empty, 0);
+      return true;
+    };
+    int prev_tile = -1;
+    for (int tile = tr.first; tile < tr.last && ok; tile += tr.step, ++ti) {
+      const int mp = tile / n_blocks, nb = tile % n_blocks;
+      const int row0 = mp * 2 * kBM + static_cast<int>(rank) * kBM + 32 * q;  // first row of this warp
       const int bs = ti & 1;
       ok = mbar_wait(&bias_full[bs], (ti >> 1) & 1, abort_flag, p.status);
+      if (ok && kMlp) ok = mbar_wait(&is_full[bs], (ti >> 1) & 1, abort_flag, p.status);
+      if (ok) ok = mbar_wait(acc_full, ti & 1, abort_flag, p.status);
       if (!ok) break;
-      const uint32_t* bias = reinterpret_cast<const uint32_t*>(smem + L::kBiasOff + bs * L::kBias) + col0 / 2;
-      if (row < p.M) {
+      tc_fence_after();
+      const uint4* bias4 = reinterpret_cast<const uint4*>(smem + L::kBiasOff + bs * L::kBias) + col0 / 8;
+      if (!kMlp) {
+        if (lane == 0) bulk_wait_group_read<0>();  // this warp's previous stores have read the staging boxes
+        __syncwarp();
+      }
+      const uint32_t ta = tmem + (static_cast<uint32_t>(32 * q) << 16) + col0;
 #pragma unroll
-        for (int v = 0; v < kBN / 16; ++v) {
-          const int n = nbase + 8 * v;
-          if (n < p.N) {
-            const uint4 bw = *reinterpret_cast<const uint4*>(bias + 4 * v);
-            const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
-            uint32_t o[4];
+      for (int c = 0; c < kBN / 64; ++c) {  // 32 columns: half of one 64-column staging box
+        uint32_t r[32];
+        tmem_ld32(ta + 32 * c, r);
+        tmem_ld_wait();
+        float yv[32];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float b0 = __uint_as_float(bb[e] << 16);
-              const float b1 = __uint_as_float(bb[e] & 0xFFFF0000u);
-              const float y0 = fmaf(__uint_as_float(r[8 * v + 2 * e]), p.out_scale, b0);
-              const float y1 = fmaf(__uint_as_float(r[8 * v + 2 * e + 1]), p.out_scale, b1);
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
-              o[e] = *reinterpret_cast<uint32_t*>(&h2);
+        for (int v = 0; v < 4; ++v) {
+          const uint4 bw = bias4[4 * c + v];
+          const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            yv[8 * v + 2 * e] = fmaf(__uint_as_float(r[8 * v + 2 * e]), p.out_scale, __uint_as_float(bb[e] << 16));
+            yv[8 * v + 2 * e + 1] =
+                fmaf(__uint_as_float(r[8 * v + 2 * e + 1]), p.out_scale, __uint_as_float(bb[e] & 0xFFFF0000u));
+          }
+        }
+        uint32_t o[16];  // this thread's 32 values of the chunk as packed bf16 (Y, or h in the MLP block)
+        if (!kMlp) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] = pack_bf16x2(yv[2 * e], yv[2 * e + 1]);
+          uint8_t* row = stg + (c >> 1) * L::kStgBox + lane * 128;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const int chunk = 4 * (c & 1) + v;  // 16-byte chunk of the 128-byte box row
+            *reinterpret_cast<uint4*>(row + ((chunk ^ (lane & 7)) << 4)) =
+                make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+          }
+        } else {
+          // h = bf16(GELU(bf16(y))), then the down layer's smoothing and NVFP4 groups of 16
+          float hv[32];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const __nv_bfloat162 yb = __floats2bfloat162_rn(yv[2 * e], yv[2 * e + 1]);
+            const float y0 = __low2float(yb), y1 = __high2float(yb);
+            const float g0 = 0.5f * y0 * (1.0f + erff(y0 * 0.70710678118654752f));
+            const float g1 = 0.5f * y1 * (1.0f + erff(y1 * 0.70710678118654752f));
+            o[e] = pack_bf16x2(g0, g1);
+            hv[2 * e] = __uint_as_float(o[e] << 16);
+            hv[2 * e + 1] = __uint_as_float(o[e] & 0xFFFF0000u);
+          }
+          const int cn = col0 + 32 * c;  // this chunk's first column within the tile
+          const float* is = reinterpret_cast<const float*>(smem + L::kIsOff + bs * L::kIs) + cn;
+          const int m = row0 + lane;
+          const int n = nb * kBN + cn;  // column of the up output = k of the down layer
+          uint32_t cw[4];
+          uint32_t sbw = 0;
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+            float v[16];
+#pragma unroll
+            for (int e = 0; e < 16; e += 4) {
+              const float4 s4 = *reinterpret_cast<const float4*>(is + 16 * g + e);
+              const float2 a = __fmul2_rn(make_float2(hv[16 * g + e], hv[16 * g + e + 1]), make_float2(s4.x, s4.y));
+              const float2 b2 =
+                  __fmul2_rn(make_float2(hv[16 * g + e + 2], hv[16 * g + e + 3]), make_float2(s4.z, s4.w));
+              v[e] = a.x;
+              v[e + 1] = a.y;
+              v[e + 2] = b2.x;
+              v[e + 3] = b2.y;
             }
-            *reinterpret_cast<uint4*>(p.Y + static_cast<size_t>(row) * p.N + n) = make_uint4(o[0], o[1], o[2], o[3]);
+            const uint32_t sb = nvfp4_quant16(v, mlp.denom, mlp.g_x, cw[2 * g], cw[2 * g + 1]);
+            sbw |= sb << (8 * g);
+          }
+          if (m < mlp.M_pad) {
+            *reinterpret_cast<uint4*>(mlp.codes + static_cast<size_t>(m) * (mlp.K >> 1) + (n >> 1)) =
+                make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            // scale-factor atom (m / 128) * (K / 64) + n / 64; the chunk's two groups are adjacent bytes
+            const size_t atom = static_cast<size_t>(m >> 7) * (mlp.K >> 6) + (n >> 6);
+            const int off = (m & 31) * 16 + ((m >> 5) & 3) * 4 + ((n >> 4) & 3);
+            *reinterpret_cast<uint16_t*>(mlp.scales + atom * 512 + off) = static_cast<uint16_t>(sbw);
+          }
+          // stage h for the T contraction: K-major 128 x 64 chunks, 128-byte swizzle
+          uint8_t* hrow = smem + L::kStgOff + (cn >> 6) * L::kHChunk + rc * 128;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const int chunk = ((cn & 63) >> 3) + v;
+            *reinterpret_cast<uint4*>(hrow + ((chunk ^ (rc & 7)) << 4)) =
+                make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
           }
         }
       }
+      tc_fence_before();
+      fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bias_empty[bs]);
+      if (lane == 0) {
+        mbar_arrive_cluster(acc_empty, 0);  // this CTA's share of TMEM is free
+        mbar_arrive(&bias_empty[bs]);
+        if (kMlp) {
+          mbar_arrive(&is_empty[bs]);
+          mbar_arrive_cluster(h_ready, 0);
+        } else {
+#pragma unroll
+          for (int b = 0; b < 2; ++b) tma_store_2d(&maps.y, stg + b * L::kStgBox, nb * kBN + col0 + 64 * b, row0);
+          bulk_commit_group();
+        }
+      }
+      // MLP: the previous tile closed a row block: its partial is complete (its
+      // contraction was committed before this tile's accumulator)
+      if (kMlp && prev_tile >= 0 && (prev_tile / n_blocks) != mp) {
+        ok = flush_t(prev_tile);
+        if (!ok) break;
+      }
+      prev_tile = tile;
+    }
+    if (kMlp && ok && prev_tile >= 0) flush_t(prev_tile);
+    if (!kMlp) {
+      if (lane == 0) bulk_wait_group<0>();  // every store of this warp has completed
+      __syncwarp();
     }
   }
 
   // ------------------------------------------------------------ teardown
+  // The leader's last commit tells both CTAs that every MMA has completed;
+  // the cluster barrier keeps each CTA alive until its partner is done
+  // signalling its barriers, then both free the pair's TMEM.
+  if (warp == 1 && leader && lane == 0) tc_commit_pair_mc(drain, 0x3);
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
-    tc_fence_after();
-    if (lane == 0) tc_commit(drain);  // arrives once every tcgen05 op issued by lane 0 has finished
-    __syncwarp();
     volatile int no_abort = 0;
     mbar_wait(drain, 0, &no_abort, nullptr);
-    tmem_dealloc(tmem, kTmemCols);
   }
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
+// T = bf16(t_scale * sum over the partial slots of each 256-row block, in slot order).
+__global__ void mlp_t_reduce_kernel(const float* tpart, int M_pad, int slots, int n_tiles, int n_blocks, int n_pairs,
+                                    float t_scale, __nv_bfloat16* T) {
+  const int mp = blockIdx.x;
+  const int t0 = mp * n_blocks, t1 = t0 + n_blocks;  // the block's tiles
+  const int p0 = mlp_first_pair(mp, n_blocks, n_tiles, n_pairs);
+  int used = 0;  // pairs whose range holds a tile of this block
+  for (int pp = p0; pp < n_pairs; ++pp) {
+    const long long f = (static_cast<long long>(pp) * n_tiles) / n_pairs;
+    const long long l = (static_cast<long long>(pp + 1) * n_tiles) / n_pairs;
+    if (f >= t1) break;
+    if (l > t0 && l > f) ++used;
+  }
+  for (int i = threadIdx.x; i < 2 * kBM * kMlpDownRP; i += blockDim.x) {
+    const int r = i / kMlpDownRP, c = i % kMlpDownRP;
+    const int m = mp * 2 * kBM + r;
+    if (m >= M_pad) continue;
+    float acc = 0.f;
+    for (int sl = 0; sl < used && sl < slots; ++sl)
+      acc += tpart[((static_cast<size_t>(mp) * slots + sl) * (2 * kBM) + r) * kMlpDownRP + c];
+    T[static_cast<size_t>(m) * kMlpDownRP + c] = __float2bfloat16_rn(acc * t_scale);
+  }
+}
+
+int max_pairs_on_device() {
+  static std::atomic<int> max_pairs_by_dev[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 74;
+  }
+  int max_pairs = (dev >= 0 && dev < 64) ? max_pairs_by_dev[dev].load() : 0;
+  if (max_pairs <= 0) {
+    cudaFuncSetAttribute(gemm_nvfp4_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         SmemNv<false>::kTotal);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = SmemNv<false>::kTotal;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, gemm_nvfp4_kernel<false>, &cfg) != cudaSuccess || clusters < 1) {
+      cudaGetLastError();
+      int sms = 148;
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      clusters = sms / 2;
+    }
+    max_pairs = clusters;
+    if (dev >= 0 && dev < 64) max_pairs_by_dev[dev].store(max_pairs);
+  }
+  return max_pairs;
+}
+
+template <bool kMlp>
+cudaError_t launch(const GemmParams& p, const MlpDownParams& mlp, const GemmMaps& maps, cudaStream_t stream) {
+  static std::atomic<unsigned long long> attr_done{0};
+  cudaError_t e = once_per_device(attr_done, [] {
+    return cudaFuncSetAttribute(gemm_nvfp4_kernel<kMlp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SmemNv<kMlp>::kTotal);
+  });
+  if (e != cudaSuccess) return e;
+  if (p.N_pad % kBN != 0) return cudaErrorInvalidValue;
+  const int tiles = ((p.M_pad + 255) / 256) * (p.N_pad / kBN);
+  const int pairs = nvfp4_pairs(tiles);
+  gemm_nvfp4_kernel<kMlp><<<2 * pairs, kThreads, SmemNv<kMlp>::kTotal, stream>>>(p, mlp, maps);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
+int nvfp4_pairs(int tiles) {
+  const int max_pairs = max_pairs_on_device();
+  return tiles < max_pairs ? tiles : max_pairs;
+}
+
+int nvfp4_mlp_slots(int tiles, int n_blocks, int pairs) {
+  int slots = 1;
+  const int m_blocks = tiles / n_blocks;
+  for (int mp = 0; mp < m_blocks; ++mp) {
+    const long long t0 = static_cast<long long>(mp) * n_blocks, t1 = t0 + n_blocks;
+    int used = 0;
+    for (int pp = mlp_first_pair(mp, n_blocks, tiles, pairs); pp < pairs; ++pp) {
+      const long long f = (static_cast<long long>(pp) * tiles) / pairs;
+      const long long l = (static_cast<long long>(pp + 1) * tiles) / pairs;
+      if (f >= t1) break;
+      if (l > t0 && l > f) ++used;
+    }
+    slots = used > slots ? used : slots;
+  }
+  return slots;
+}
 
 cudaError_t launch_gemm_nvfp4(const GemmParams& p, const GemmMaps& maps, cudaStream_t stream) {
-  static std::atomic<unsigned long long> attr_done{0};
-  cudaError_t e = once_per_device(attr_done, [] {
-    return cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SmemNv::kTotal);
-  });
-  if (e != cudaSuccess) return e;
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
-  const int tiles = (p.M_pad / kBM) * ((p.N + kBN - 1) / kBN);
-  const int grid = tiles < sms ? tiles : sms;
-  gemm_nvfp4_kernel<<<grid, kThreads, SmemNv::kTotal, stream>>>(p, maps);
+  return launch<false>(p, MlpDownParams{}, maps, stream);
+}
+
+cudaError_t launch_gemm_nvfp4_mlp(const GemmParams& p, const MlpDownParams& mlp, const GemmMaps& maps,
+                                  cudaStream_t stream) {
+  if (!mlp.codes || !mlp.scales || !mlp.tpart || !mlp.inv_s || mlp.K != p.N || mlp.M_pad < p.M_pad)
+    return cudaErrorInvalidValue;
+  return launch<true>(p, mlp, maps, stream);
+}
+
+cudaError_t launch_mlp_t_reduce(const float* tpart, int M_pad, int slots, int tiles, int n_blocks, int pairs,
+                                float t_scale, __nv_bfloat16* T, cudaStream_t stream) {
+  const int m_blocks = (M_pad + 255) / 256;
+  mlp_t_reduce_kernel<<<m_blocks, 256, 0, stream>>>(tpart, M_pad, slots, tiles, n_blocks, pairs, t_scale, T);
   return cudaGetLastError();
 }
 

@@ -67,11 +67,42 @@ struct GemmParams {
   int* status;                 // device status word (kDevTimeout on a given-up wait)
 };
 struct GemmMaps {
-  CUtensorMap a;   // activation codes
-  CUtensorMap b;   // weight codes
-  CUtensorMap t;   // T [M_pad, RP] bf16
-  CUtensorMap l2;  // L2T [N_pad, RP] bf16
+  CUtensorMap a;    // activation codes
+  CUtensorMap b;    // weight codes
+  CUtensorMap t;    // T [M_pad, RP] bf16
+  CUtensorMap l2;   // L2T [N_pad, RP] bf16
+  CUtensorMap sfa;  // NVFP4 activation scale-factor atoms as uint32 [atoms, 128], box {128, 4}
+  CUtensorMap sfb;  // NVFP4 weight scale-factor atoms, same view
+  CUtensorMap y;    // NVFP4: Y [M, N] bf16, box {64, 32}, 128-byte swizzle (TMA stores)
+  CUtensorMap l1h_down;  // MLP block: the down layer's L1s^T high part [RP_down, K_down], box {64, RP_down / 2}
+  CUtensorMap l1l_down;  // ... and low part
 };
+
+// The down layer of an MLP block as the fused epilogue of the up layer's
+// NVFP4 GEMM sees it: GELU of the up output is smoothed and quantized
+// straight into the down layer's activation buffers, and its branch input T
+// is accumulated from the same tile (partials over the pairs of SMs, summed
+// by nvfp4_mlp_t_reduce).
+constexpr int kMlpDownRP = 32;  // branch width of the down layer the fused epilogue supports
+struct MlpDownParams {
+  int K;                 // the down layer's K (= the up layer's N)
+  int M_pad;             // rows of the down layer's activation buffers
+  const float* inv_s;    // [K]
+  uint8_t* codes;        // [M_pad, K/2] packed E2M1
+  uint8_t* scales;       // scale-factor atoms [M_pad/128][K/64][512]
+  float g_x, denom;      // the down layer's static activation tensor scale and fp32(6 g_x)
+  float* tpart;          // T partials [ceil(M_pad / 256)][slots][256][kMlpDownRP] float
+  int slots;             // partial slots per 256-row block
+};
+// Pairs of SMs the NVFP4 GEMM runs on for `tiles` 256 x 256 tiles (current device).
+int nvfp4_pairs(int tiles);
+// Partial slots per 256-row block the fused MLP epilogue needs with `pairs` pairs.
+int nvfp4_mlp_slots(int tiles, int n_blocks, int pairs);
+cudaError_t launch_gemm_nvfp4_mlp(const GemmParams& p, const MlpDownParams& mlp, const GemmMaps& maps,
+                                  cudaStream_t stream);
+// T = bf16(t_scale * sum of the partials in slot order) [M_pad, kMlpDownRP].
+cudaError_t launch_mlp_t_reduce(const float* tpart, int M_pad, int slots, int tiles, int n_blocks, int pairs,
+                                float t_scale, __nv_bfloat16* T, cudaStream_t stream);
 // Rows of one TMA box of the weight codes, of L2^T and of the activation codes.
 // The GEMMs load a tile's operand rows as several boxes: copies in flight,
 // not their size, set the TMA throughput of an SM.

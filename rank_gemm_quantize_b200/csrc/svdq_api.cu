@@ -83,7 +83,7 @@ struct MapCache {
   struct Entry {
     const void* key = nullptr;
     int rows = -1;
-    CUtensorMap a{}, b{};
+    CUtensorMap a{}, b{}, c{};
   };
   Entry e[N];
   int next = 0;
@@ -144,9 +144,13 @@ struct svdq_layer {
   void* wscales = nullptr;       // INT4 float [K/64][N_pad]; NVFP4 atoms [N_pad/128][K/64][512]
   int* status = nullptr;         // device status word
   int* k1_counters = nullptr;    // activation-kernel arrival counters per 128-row block (zero between launches)
-  CUtensorMap map_b{}, map_l2{}, map_l1h{}, map_l1l{};
+  CUtensorMap map_b{}, map_l2{}, map_l1h{}, map_l1l{}, map_sfb{};
+  // as the down layer of a fused MLP block: L1s^T hi / lo with 16-row boxes
+  CUtensorMap map_l1h_half{}, map_l1l_half{};
+  bool mlp_maps_ready = false;
   MapCache<8> ws_maps;  // (workspace, M) -> activation codes map (a), T map (b)
   MapCache<8> x_maps;   // (X, M) -> X map (a)
+  MapCache<8> y_maps;   // (Y, M) -> Y map (a), NVFP4 only
 };
 
 namespace {
@@ -237,12 +241,21 @@ void free_layer(svdq_layer* h) {
   delete h;
 }
 
+// NVFP4 scale-factor atoms (512 bytes each) as a uint32 [atoms, 128] tensor,
+// loaded four atoms (the four 64-wide k-blocks of a 256-deep k-tile) at a time.
+bool make_sf_map(CUtensorMap* m, const void* base, uint64_t atoms) {
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, base, 128, atoms, 512, 128, 4, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 svdq_status build_static_maps(svdq_layer* h) {
   const bool i4 = h->fmt == SVDQ_INT4_G64;
   const uint64_t row = i4 ? h->K : h->K / 2;
   if (!make_map(&h->map_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, row, h->N_pad, row, 128, kWeightBoxRows,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (weight codes) failed");
+  h->map_sfb = CUtensorMap{};
+  if (!i4 && !make_sf_map(&h->map_sfb, h->wscales, static_cast<uint64_t>(h->N_pad / 128) * (h->K / 64)))
+    return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (weight scale factors) failed");
   h->map_l2 = CUtensorMap{};
   h->map_l1h = CUtensorMap{};
   h->map_l1l = CUtensorMap{};
@@ -258,6 +271,8 @@ svdq_status build_static_maps(svdq_layer* h) {
   }
   h->ws_maps.clear();
   h->x_maps.clear();
+  h->y_maps.clear();
+  h->mlp_maps_ready = false;
   return SVDQ_OK;
 }
 
@@ -679,6 +694,70 @@ svdq_status svdq_workspace_size(svdq_layer_t h, int M, size_t* bytes) {
 
 namespace {
 
+// The GEMM of a forward on activations already in the layer's layouts
+// (codes, scales, T for M rows). With mlp set (NVFP4 only) the GEMM is the up
+// layer of an MLP block: its epilogue writes the down layer's activations
+// instead of Y.
+svdq_status gemm_stage(svdq_layer* h, int M, void* Y, uint8_t* codes, void* scales, __nv_bfloat16* T,
+                       const MlpDownParams* mlp, const GemmMaps* mlp_maps, cudaStream_t st) {
+  const int M_pad = round_up(M, 128);
+  auto* we = h->ws_maps.find(codes, M);
+  if (!we) {
+    we = h->ws_maps.insert(codes, M);
+    const bool i4 = h->fmt == SVDQ_INT4_G64;
+    const uint64_t row = i4 ? h->K : h->K / 2;
+    we->b = CUtensorMap{};
+    we->c = CUtensorMap{};
+    if (!make_map(&we->a, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, row, M_pad, row, 128, kActBoxRows,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        (!i4 && !make_sf_map(&we->c, scales, static_cast<uint64_t>(M_pad / 128) * (h->K / 64))) ||
+        (h->RP > 0 && !make_map(&we->b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, h->RP, M_pad,
+                                static_cast<uint64_t>(h->RP) * 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))) {
+      we->key = nullptr;
+      return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (activations) failed");
+    }
+  }
+  GemmParams p{};
+  p.M = M;
+  p.N = h->N;
+  p.K = h->K;
+  p.RP = h->RP;
+  p.Y = static_cast<__nv_bfloat16*>(Y);
+  p.bias = h->bias;
+  p.sa = scales;
+  p.sb = h->wscales;
+  p.M_pad = M_pad;
+  p.N_pad = h->N_pad;
+  p.out_scale = h->gxgw;
+  p.status = h->status;
+  GemmMaps maps = mlp_maps ? *mlp_maps : GemmMaps{};
+  maps.a = we->a;
+  maps.b = h->map_b;
+  maps.t = we->b;
+  maps.l2 = h->map_l2;
+  maps.sfa = we->c;
+  maps.sfb = h->map_sfb;
+  if (h->fmt == SVDQ_NVFP4_G16 && !mlp) {
+    auto* ye = h->y_maps.find(Y, M);
+    if (!ye) {
+      ye = h->y_maps.insert(Y, M);
+      if (!make_map(&ye->a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, h->N, M, static_cast<uint64_t>(h->N) * 2, 64, 32,
+                    CU_TENSOR_MAP_SWIZZLE_128B)) {
+        ye->key = nullptr;
+        return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (Y) failed");
+      }
+    }
+    maps.y = ye->a;
+  }
+  cudaError_t ce;
+  if (mlp)
+    ce = launch_gemm_nvfp4_mlp(p, *mlp, maps, st);
+  else
+    ce = h->fmt == SVDQ_INT4_G64 ? launch_gemm_int4(p, maps, st) : launch_gemm_nvfp4(p, maps, st);
+  if (ce != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("GEMM kernel: ") + cudaGetErrorString(ce));
+  return SVDQ_OK;
+}
+
 svdq_status forward_impl(svdq_layer* h, const void* X, int M, void* Y, void* workspace, size_t ws_bytes,
                          const uint32_t* row_mask, void* stream, void* const* events) {
   if (check_layer(h)) return SVDQ_ERR_INVALID_ARG;
@@ -700,41 +779,99 @@ svdq_status forward_impl(svdq_layer* h, const void* X, int M, void* Y, void* wor
   svdq_status e = launch_k1(h, X, M, codes, scales, T, Tpart, w, row_mask, st);
   if (e) return e;
   if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[1]), st));
-  auto* we = h->ws_maps.find(workspace, M);
-  if (!we) {
-    we = h->ws_maps.insert(workspace, M);
-    const bool i4 = h->fmt == SVDQ_INT4_G64;
-    const uint64_t row = i4 ? h->K : h->K / 2;
-    we->b = CUtensorMap{};
-    if (!make_map(&we->a, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, row, w.M_pad, row, 128, kActBoxRows,
-                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-        (h->RP > 0 && !make_map(&we->b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T, h->RP, w.M_pad,
-                                static_cast<uint64_t>(h->RP) * 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))) {
-      we->key = nullptr;
-      return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (activations) failed");
-    }
-  }
-  GemmParams p{};
-  p.M = M;
-  p.N = h->N;
-  p.K = h->K;
-  p.RP = h->RP;
-  p.Y = static_cast<__nv_bfloat16*>(Y);
-  p.bias = h->bias;
-  p.sa = scales;
-  p.sb = h->wscales;
-  p.M_pad = w.M_pad;
-  p.N_pad = h->N_pad;
-  p.out_scale = h->gxgw;
-  p.status = h->status;
-  GemmMaps maps;
-  maps.a = we->a;
-  maps.b = h->map_b;
-  maps.t = we->b;
-  maps.l2 = h->map_l2;
-  cudaError_t ce = h->fmt == SVDQ_INT4_G64 ? launch_gemm_int4(p, maps, st) : launch_gemm_nvfp4(p, maps, st);
-  if (ce != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("GEMM kernel: ") + cudaGetErrorString(ce));
+  if ((e = gemm_stage(h, M, Y, codes, scales, T, nullptr, nullptr, st))) return e;
   if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[2]), st));
+  return SVDQ_OK;
+}
+
+// Workspace of an MLP block forward: the up layer's forward workspace, the
+// down layer's activation codes, scales and T, and the T partials.
+struct MlpLayout {
+  WsLayout up, down;
+  size_t down_off, tpart_off, total;
+  int tiles, n_blocks, pairs, slots;
+};
+
+MlpLayout mlp_layout(const svdq_layer* up, const svdq_layer* down, int M) {
+  MlpLayout l{};
+  l.up = ws_layout(up, M);
+  l.down = ws_layout(down, M);
+  l.down_off = align256(l.up.total);
+  l.tpart_off = l.down_off + align256(l.down.Tpart);  // the down layer's codes, scales and T only
+  l.n_blocks = up->N_pad / 256;
+  l.tiles = ((l.up.M_pad + 255) / 256) * l.n_blocks;
+  l.pairs = nvfp4_pairs(l.tiles);
+  l.slots = nvfp4_mlp_slots(l.tiles, l.n_blocks, l.pairs);
+  const size_t tpart = static_cast<size_t>((l.up.M_pad + 255) / 256) * l.slots * 256 * kMlpDownRP * 4;
+  l.total = l.tpart_off + align256(tpart);
+  return l;
+}
+
+svdq_status check_mlp(svdq_layer* up, svdq_layer* down) {
+  if (!up || !down) return fail(SVDQ_ERR_INVALID_ARG, "layer is NULL");
+  if (up->fmt != SVDQ_NVFP4_G16 || down->fmt != SVDQ_NVFP4_G16)
+    return fail(SVDQ_ERR_UNSUPPORTED, "the fused MLP block needs two NVFP4 layers");
+  if (up->N != down->K) return fail(SVDQ_ERR_INVALID_ARG, "the up layer's N must be the down layer's K");
+  if (down->K % 256) return fail(SVDQ_ERR_UNSUPPORTED, "the fused MLP block needs the down layer's K % 256 == 0");
+  if (down->RP != kMlpDownRP)
+    return fail(SVDQ_ERR_UNSUPPORTED, "the fused MLP block needs a down-layer branch of 1..32 columns");
+  if (up->device != down->device) return fail(SVDQ_ERR_INVALID_ARG, "the layers live on different devices");
+  return SVDQ_OK;
+}
+
+svdq_status mlp_impl(svdq_layer* up, svdq_layer* down, const void* X, int M, void* Y, void* workspace,
+                     size_t ws_bytes, void* stream, void* const* events) {
+  if (svdq_status e = check_mlp(up, down)) return e;
+  if (!X || !Y || !workspace || M < 1) return fail(SVDQ_ERR_INVALID_ARG, "NULL pointer or M < 1");
+  if (!aligned16(X) || !aligned16(Y) || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return fail(SVDQ_ERR_INVALID_ARG, "X/Y must be 16-byte and the workspace 256-byte aligned");
+  if (svdq_status e = check_layer_device(up)) return e;
+  const MlpLayout l = mlp_layout(up, down, M);
+  if (ws_bytes < l.total) return fail(SVDQ_ERR_INVALID_ARG, "workspace too small");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  uint8_t* dbase = base + l.down_off;
+  uint8_t* codes_d = dbase + l.down.codes;
+  uint8_t* scales_d = dbase + l.down.scales;
+  __nv_bfloat16* T_d = reinterpret_cast<__nv_bfloat16*>(dbase + l.down.T);
+  float* tpart = reinterpret_cast<float*>(base + l.tpart_off);
+  // the down layer's factor as the fused epilogue loads it: each CTA of a pair its 16 rows
+  if (!down->mlp_maps_ready) {
+    if (!make_map(&down->map_l1h_half, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, down->L1sTh, down->K, down->RP,
+                  static_cast<uint64_t>(down->K) * 2, 64, kMlpDownRP / 2, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&down->map_l1l_half, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, down->L1sTl, down->K, down->RP,
+                  static_cast<uint64_t>(down->K) * 2, 64, kMlpDownRP / 2, CU_TENSOR_MAP_SWIZZLE_128B))
+      return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (down-layer factor) failed");
+    down->mlp_maps_ready = true;
+  }
+  if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[0]), st));
+  svdq_status e = launch_k1(up, X, M, base + l.up.codes, base + l.up.scales,
+                            reinterpret_cast<__nv_bfloat16*>(base + l.up.T), reinterpret_cast<float*>(base + l.up.Tpart),
+                            l.up, nullptr, st);
+  if (e) return e;
+  if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[1]), st));
+  MlpDownParams mp{};
+  mp.K = down->K;
+  mp.M_pad = l.down.M_pad;
+  mp.inv_s = down->inv_s;
+  mp.codes = codes_d;
+  mp.scales = scales_d;
+  mp.g_x = down->g_x;
+  mp.denom = down->denom;
+  mp.tpart = tpart;
+  mp.slots = l.slots;
+  GemmMaps extra{};
+  extra.l1h_down = down->map_l1h_half;
+  extra.l1l_down = down->map_l1l_half;
+  if ((e = gemm_stage(up, M, nullptr, base + l.up.codes, base + l.up.scales,
+                      reinterpret_cast<__nv_bfloat16*>(base + l.up.T), &mp, &extra, st)))
+    return e;
+  if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[2]), st));
+  cudaError_t ce = launch_mlp_t_reduce(tpart, l.down.M_pad, l.slots, l.tiles, l.n_blocks, l.pairs, down->t_scale, T_d, st);
+  if (ce != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("T reduction: ") + cudaGetErrorString(ce));
+  if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[3]), st));
+  if ((e = gemm_stage(down, M, Y, codes_d, scales_d, T_d, nullptr, nullptr, st))) return e;
+  if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[4]), st));
   return SVDQ_OK;
 }
 
@@ -745,6 +882,36 @@ extern "C" {
 svdq_status svdq_linear_forward(svdq_layer_t h, const void* X, int M, void* Y, void* workspace, size_t ws_bytes,
                                 void* stream) {
   return forward_impl(h, X, M, Y, workspace, ws_bytes, nullptr, stream, nullptr);
+}
+
+svdq_status svdq_mlp_workspace_size(svdq_layer_t up, svdq_layer_t down, int M, size_t* bytes) {
+  if (svdq_status e = check_mlp(up, down)) return e;
+  if (!bytes || M < 1) return fail(SVDQ_ERR_INVALID_ARG, "bad workspace query");
+  *bytes = mlp_layout(up, down, M).total;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_mlp_workspace_layout(svdq_layer_t up, svdq_layer_t down, int M, size_t* offsets) {
+  if (svdq_status e = check_mlp(up, down)) return e;
+  if (!offsets || M < 1) return fail(SVDQ_ERR_INVALID_ARG, "bad layout query");
+  const MlpLayout l = mlp_layout(up, down, M);
+  offsets[0] = l.down_off + l.down.codes;
+  offsets[1] = l.down_off + l.down.scales;
+  offsets[2] = l.down_off + l.down.T;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_mlp_forward(svdq_layer_t up, svdq_layer_t down, const void* X, int M, void* Y, void* workspace,
+                             size_t ws_bytes, void* stream) {
+  return mlp_impl(up, down, X, M, Y, workspace, ws_bytes, stream, nullptr);
+}
+
+svdq_status svdq_mlp_forward_profiled(svdq_layer_t up, svdq_layer_t down, const void* X, int M, void* Y,
+                                      void* workspace, size_t ws_bytes, void* stream, void* const* events) {
+  if (!events) return fail(SVDQ_ERR_INVALID_ARG, "five events needed");
+  for (int i = 0; i < 5; ++i)
+    if (!events[i]) return fail(SVDQ_ERR_INVALID_ARG, "five events needed");
+  return mlp_impl(up, down, X, M, Y, workspace, ws_bytes, stream, events);
 }
 
 svdq_status svdq_linear_forward_masked(svdq_layer_t h, const void* X, int M, void* Y, void* workspace,

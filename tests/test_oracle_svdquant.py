@@ -466,3 +466,34 @@ def test_weight_only_is_exact_on_representable_weights():
     p = S.prepare_weight_only(W, b)
     assert np.array_equal(S.dequantize_weight_only(p), W.T)
     assert np.array_equal(S.forward_weight_only(p, X), X @ W + b)
+
+
+# ------------------------------------------------------------- the MLP block
+
+def test_gelu_closed_forms():
+    x = np.array([0.0, 1.0, -1.0, 3.0, -3.0, 10.0, -10.0, 0.5])
+    g = S.gelu_erf(x)
+    assert g[0] == 0.0
+    # GELU(x) - GELU(-x) = x exactly in the definition (Phi(x) + Phi(-x) = 1)
+    assert np.allclose(g[1::2][:3] - g[2::2][:3], x[1::2][:3], rtol=0, atol=1e-15)
+    assert abs(g[5] - 10.0) < 1e-20 and abs(g[6]) < 1e-20  # the tails
+    assert abs(g[1] - 0.8413447460685429) < 1e-15  # Phi(1) = 0.8413447460685429...
+    assert abs(g[7] - 0.5 * 0.6914624612740131) < 1e-15  # Phi(0.5)
+
+
+def test_mlp_block_is_the_composition_of_two_brute_force_layers():
+    """The block against two plain-loop layers with GELU between them (math.erf)."""
+    up_l = workloads.custom(3, 128, 64, 2, "nvfp4_g16", seed=49, n_outliers=2)
+    X, Wu, bu = workloads.to_f64(up_l.X), workloads.to_f64(up_l.W), workloads.to_f64(up_l.bias)
+    rng = np.random.Generator(np.random.PCG64(50))
+    Wd = F.bf16_round(rng.normal(0, 0.02, (64, 16)))
+    bd = F.bf16_round(rng.normal(0, 0.01, 16))
+    p_up = S.prepare(Wu, bu, S.calibrate_absmax(X), "nvfp4_g16", 0.5, 2)
+    y_up = F.bf16_round(_brute_force_layer(X, Wu, bu, S.calibrate_absmax(X), "nvfp4_g16", 2, p_up.L1, p_up.L2))
+    h = F.bf16_round(np.array([[0.5 * v * (1 + math.erf(v / math.sqrt(2))) for v in row] for row in y_up]))
+    a_d = S.calibrate_absmax(h)
+    p_down = S.prepare(Wd, bd, a_d, "nvfp4_g16", 0.5, 2)
+    want = _brute_force_layer(h, Wd, bd, a_d, "nvfp4_g16", 2, p_down.L1, p_down.L2)
+    r = S.mlp_forward(p_up, p_down, X)
+    assert np.array_equal(r.y_up, y_up) and np.array_equal(r.h, h)
+    assert np.allclose(r.down.Y, want, rtol=1e-12, atol=1e-12)
