@@ -171,13 +171,17 @@ SVDQ_API svdq_status svdq_linear_forward_profiled(svdq_layer_t layer, const void
 
 /* The MLP block of two layers, Y = down(GELU(up(X))), fused across the
  * boundary between them: the up layer's GEMM epilogue rounds its output to
- * bf16, applies GELU (the erf form, in float32) and rounds to bf16 (h, what a
- * plain composition of the layers would pass on), then smooths and quantizes
+ * bf16, applies GELU (the erf form in float32, erf by Abramowitz & Stegun
+ * 7.1.26, absolute error under 1e-6) and rounds to bf16 (h, what a plain
+ * composition of the layers would pass on), then smooths and quantizes
  * h for the down layer straight into the down layer's activation codes and
  * scales, and contracts it with the down layer's factor for the down layer's
  * branch input T. h itself never goes to device memory. Abstract: the
  * low-rank branch is fused into the low-bit kernels to cut redundant memory
- * traffic; this carries that across the two layers of the block.
+ * traffic; this carries that across the two layers of the block. The up
+ * layer's branch input T is carried as a bf16 pair here (about 16 significant
+ * bits, where a single forward holds it in bf16), because the bf16 rounding
+ * of the up output decides the down layer's codes.
  * Kernels on `stream`: the up layer's activation kernel, the fused up GEMM, a
  * small fixed-order sum of the T partials, the down layer's GEMM.
  *   up, down  NVFP4 layers on the same device, up->N == down->K,

@@ -160,7 +160,7 @@ __device__ __forceinline__ bool column_on(const ActQuantParams& p, uint32_t mask
 }
 
 // Stores 8 consecutive T columns c0 .. c0+7 of row r (scaled by t_scale, the
-// columns of unselected adapters zeroed).
+// columns of unselected adapters zeroed); with T_lo also the bf16 remainders.
 __device__ __forceinline__ void store_t8(const ActQuantParams& p, int RP, int r, int c0, const float (&a)[8]) {
   float v[8];
   // the mask has one entry per row of X; padding rows (r >= M) hold zeros anyway
@@ -170,7 +170,16 @@ __device__ __forceinline__ void store_t8(const ActQuantParams& p, int RP, int r,
   for (int e = 0; e < 8; ++e) v[e] = (masked && !column_on(p, mask, c0 + e)) ? 0.f : a[e] * p.t_scale;
   const uint4 o = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
                              pack_bf16x2(v[6], v[7]));
-  *reinterpret_cast<uint4*>(p.T + static_cast<size_t>(r) * RP + c0) = o;
+  const size_t off = static_cast<size_t>(r) * RP + c0;
+  *reinterpret_cast<uint4*>(p.T + off) = o;
+  if (p.T_lo) {
+    const uint32_t w[4] = {o.x, o.y, o.z, o.w};
+    uint32_t l[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      l[e] = pack_bf16x2(v[2 * e] - __uint_as_float(w[e] << 16), v[2 * e + 1] - __uint_as_float(w[e] & 0xFFFF0000u));
+    *reinterpret_cast<uint4*>(p.T_lo + off) = make_uint4(l[0], l[1], l[2], l[3]);
+  }
 }
 
 template <int FMT, int RP>

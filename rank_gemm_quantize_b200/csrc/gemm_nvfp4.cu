@@ -37,7 +37,10 @@
 //           tile's MMAs start) and stores its two 32 x 64 boxes with TMA
 //           (rows and columns past M and N are clipped by the tensor map).
 //
-// MLP-block variant (kMlp, the up layer of up -> GELU -> down): the epilogue
+// MLP-block variant (kMlp, the up layer of up -> GELU -> down): the branch
+// reads T as a bf16 pair (T + T_lo, about 16 significant bits), so the up
+// output, and with it the bf16 rounding of its GELU that decides the down
+// layer's codes, matches the exact product far more closely. The epilogue
 // does not store Y. It rounds the output to bf16, applies GELU (erf form,
 // float32) and rounds to bf16 (h: the tensor a plain composition of the two
 // layers would pass on), then smooths and NVFP4-quantizes h for the down
@@ -96,6 +99,7 @@ static_assert(SmemNv<false>::kTotal <= 232448 && SmemNv<true>::kTotal <= 232448,
 static_assert(SmemNv<false>::kStage % 1024 == 0 && SmemNv<true>::kStgOff % 1024 == 0 &&
                   SmemNv<false>::kStgOff % 1024 == 0 && SmemNv<true>::kL1Off % 1024 == 0,
               "swizzled tiles start 1 KB-aligned");
+static_assert(2 * kBM * 64 <= SmemNv<true>::kA, "T and its low part share a stage's A slot");
 static_assert(kBNHalf == kWeightBoxRows && kBM == kActBoxRows, "each CTA loads one box per operand");
 
 // TMEM columns (each CTA): accumulator [0, 256), then one scale-factor slot per
@@ -115,6 +119,24 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// GELU(y) = y Phi(y) = 0.5 y (1 + erf(y / sqrt 2)), with erf by the rational
+// approximation of Abramowitz and Stegun, Handbook of Mathematical Functions,
+// formula 7.1.26: for x >= 0, erfc(x) ~ t (a1 + t (a2 + t (a3 + t (a4 + t a5))))
+// exp(-x^2), t = 1 / (1 + p x), absolute error at most 1.5e-7. The negative
+// side uses 1 + erf(-x) = erfc(x) directly, so no cancellation; with the
+// float32 evaluation the result is within about 5e-7 of 1 + erf, absolute.
+// The same instructions on every lane (no branch on the argument).
+__device__ __forceinline__ float gelu(float y) {
+  const float x = fabsf(y) * 0.70710678118654752f;
+  const float t = __fdividef(1.0f, fmaf(0.3275911f, x, 1.0f));
+  float poly = fmaf(1.061405429f, t, -1.453152027f);
+  poly = fmaf(poly, t, 1.421413741f);
+  poly = fmaf(poly, t, -0.284496736f);
+  poly = fmaf(poly, t, 0.254829592f);
+  const float erfc_x = poly * t * __expf(-x * x);
+  return 0.5f * y * (y >= 0.f ? 2.0f - erfc_x : erfc_x);
+}
+
 // The tile range of pair `pair`: round-robin for the plain GEMM (the pairs in
 // flight share the weight panel in L2); contiguous in row-major tile order for
 // the MLP variant (the down layer's T accumulates over a row block).
@@ -130,12 +152,27 @@ __device__ __forceinline__ TileRange tile_range(int pair, int n_pairs, int n_til
   return {pair, n_tiles, n_pairs};
 }
 
-// The first pair whose contiguous range holds a tile of 256-row block mp.
+// The first pair whose contiguous range holds a tile of 256-row block mp: the
+// smallest p with floor((p + 1) n_tiles / n_pairs) > t for the block's first
+// tile t, i.e. p = ceil((t + 1) n_pairs / n_tiles) - 1.
 __host__ __device__ inline int mlp_first_pair(int mp, int n_blocks, int n_tiles, int n_pairs) {
   const long long t = static_cast<long long>(mp) * n_blocks;
-  int p = 0;
-  while (p < n_pairs - 1 && (static_cast<long long>(p + 1) * n_tiles) / n_pairs <= t) ++p;
-  return p;
+  const long long p = ((t + 1) * n_pairs + n_tiles - 1) / n_tiles - 1;
+  return static_cast<int>(p < 0 ? 0 : (p > n_pairs - 1 ? n_pairs - 1 : p));
+}
+
+// The number of pairs whose ranges hold tiles of row block mp (the partial
+// slots it uses).
+__host__ __device__ inline int mlp_block_pairs(int mp, int n_blocks, int n_tiles, int n_pairs) {
+  const long long t0 = static_cast<long long>(mp) * n_blocks, t1 = t0 + n_blocks;
+  int used = 0;
+  for (int pp = mlp_first_pair(mp, n_blocks, n_tiles, n_pairs); pp < n_pairs; ++pp) {
+    const long long f = (static_cast<long long>(pp) * n_tiles) / n_pairs;
+    const long long l = (static_cast<long long>(pp + 1) * n_tiles) / n_pairs;
+    if (f >= t1) break;
+    if (l > t0 && l > f) ++used;
+  }
+  return used;
 }
 
 template <bool kMlp>
@@ -227,6 +264,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (kMlp) {
         prefetch_tensormap(&maps.l1h_down);
         prefetch_tensormap(&maps.l1l_down);
+        if (n_lr > 0) prefetch_tensormap(&maps.t_lo);
       }
       bool ok = true;
       int it = 0;          // k-tiles issued over all tiles of this CTA
@@ -265,9 +303,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               tma_load_2d_pair(st + L::kA + L::kB + L::kSfa + h * 2048, &maps.sfb, fb, 0,
                                (nb * (kBN / 128) + h) * kb_total + kb0);
           } else {
-            if (leader) mbar_arrive_expect_tx(&full[s], 2 * (kBM * 64 + kBNHalf * 64));
+            if (leader) mbar_arrive_expect_tx(&full[s], 2 * ((kMlp ? 2 : 1) * kBM * 64 + kBNHalf * 64));
             const int c = k - n_main;  // 32-column slice of the branch
             tma_load_2d_pair(st, &maps.t, fb, c * 32, m0);
+            if (kMlp) tma_load_2d_pair(st + kBM * 64, &maps.t_lo, fb, c * 32, m0);
             tma_load_2d_pair(st + L::kA, &maps.l2, fb, c * 32, n0 + static_cast<int>(rank) * kBNHalf);
           }
         }
@@ -369,6 +408,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const uint64_t ad = smem_desc(a_base + 32 * j, 16, 512, kSw64);
                 const uint64_t bd = smem_desc(b_base + 32 * j, 16, 512, kSw64);
                 mma_f16_pair(tmem, ad, bd, idesc_lr, 1u);
+                if (kMlp)  // T's low part: the block's GELU input carries about 16 bits of T
+                  mma_f16_pair(tmem, smem_desc(a_base + kBM * 64 + 32 * j, 16, 512, kSw64), bd, idesc_lr, 1u);
               }
             }
             tc_commit_pair_mc(&empty[s], 0x3);  // the stage is free in both CTAs
@@ -470,101 +511,108 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         __syncwarp();
       }
       const uint32_t ta = tmem + (static_cast<uint32_t>(32 * q) << 16) + col0;
+      // Phase A: the accumulator -> y = out_scale acc + b, bf16, into the staging buffer (the Y
+      // boxes; in the MLP block the K-major h chunks, where phase B turns y into h in place)
 #pragma unroll
       for (int c = 0; c < kBN / 64; ++c) {  // 32 columns: half of one 64-column staging box
         uint32_t r[32];
         tmem_ld32(ta + 32 * c, r);
         tmem_ld_wait();
-        float yv[32];
+        uint32_t o[16];  // this thread's 32 values of the chunk as packed bf16
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           const uint4 bw = bias4[4 * c + v];
           const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            yv[8 * v + 2 * e] = fmaf(__uint_as_float(r[8 * v + 2 * e]), p.out_scale, __uint_as_float(bb[e] << 16));
-            yv[8 * v + 2 * e + 1] =
-                fmaf(__uint_as_float(r[8 * v + 2 * e + 1]), p.out_scale, __uint_as_float(bb[e] & 0xFFFF0000u));
-          }
+          for (int e = 0; e < 4; ++e)
+            o[4 * v + e] =
+                pack_bf16x2(fmaf(__uint_as_float(r[8 * v + 2 * e]), p.out_scale, __uint_as_float(bb[e] << 16)),
+                            fmaf(__uint_as_float(r[8 * v + 2 * e + 1]), p.out_scale,
+                                 __uint_as_float(bb[e] & 0xFFFF0000u)));
         }
-        uint32_t o[16];  // this thread's 32 values of the chunk as packed bf16 (Y, or h in the MLP block)
+        uint8_t* row;
+        int chunk0;
+        if (!kMlp) {
+          row = stg + (c >> 1) * L::kStgBox + lane * 128;
+          chunk0 = 4 * (c & 1);
+        } else {
+          const int cn = col0 + 32 * c;
+          row = smem + L::kStgOff + (cn >> 6) * L::kHChunk + rc * 128;
+          chunk0 = (cn & 63) >> 3;
+        }
+        const int sw = kMlp ? (rc & 7) : (lane & 7);
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          *reinterpret_cast<uint4*>(row + (((chunk0 + v) ^ sw) << 4)) =
+              make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+      }
+      tc_fence_before();
+      if (!kMlp) fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_cluster(acc_empty, 0);  // this CTA's share of TMEM is free: the next tile's MMAs start
+        mbar_arrive(&bias_empty[bs]);
         if (!kMlp) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) o[e] = pack_bf16x2(yv[2 * e], yv[2 * e + 1]);
-          uint8_t* row = stg + (c >> 1) * L::kStgBox + lane * 128;
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const int chunk = 4 * (c & 1) + v;  // 16-byte chunk of the 128-byte box row
-            *reinterpret_cast<uint4*>(row + ((chunk ^ (lane & 7)) << 4)) =
-                make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
-          }
-        } else {
-          // h = bf16(GELU(bf16(y))), then the down layer's smoothing and NVFP4 groups of 16
-          float hv[32];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const __nv_bfloat162 yb = __floats2bfloat162_rn(yv[2 * e], yv[2 * e + 1]);
-            const float y0 = __low2float(yb), y1 = __high2float(yb);
-            const float g0 = 0.5f * y0 * (1.0f + erff(y0 * 0.70710678118654752f));
-            const float g1 = 0.5f * y1 * (1.0f + erff(y1 * 0.70710678118654752f));
-            o[e] = pack_bf16x2(g0, g1);
-            hv[2 * e] = __uint_as_float(o[e] << 16);
-            hv[2 * e + 1] = __uint_as_float(o[e] & 0xFFFF0000u);
-          }
-          const int cn = col0 + 32 * c;  // this chunk's first column within the tile
-          const float* is = reinterpret_cast<const float*>(smem + L::kIsOff + bs * L::kIs) + cn;
-          const int m = row0 + lane;
-          const int n = nb * kBN + cn;  // column of the up output = k of the down layer
-          uint32_t cw[4];
+          for (int b = 0; b < 2; ++b) tma_store_2d(&maps.y, stg + b * L::kStgBox, nb * kBN + col0 + 64 * b, row0);
+          bulk_commit_group();
+        }
+      }
+      if (kMlp) {
+        // Phase B, overlapping the next tile's mainloop: h = bf16(GELU(y)) in place, then the down
+        // layer's smoothing and NVFP4 groups of 16; this thread's row, 64 columns at a time
+        const float* is_tile = reinterpret_cast<const float*>(smem + L::kIsOff + bs * L::kIs);
+        const int m = row0 + lane;
+#pragma unroll 1
+        for (int piece = 0; piece < 2; ++piece) {
+          const int cn = col0 + 64 * piece;  // first column of the 64 within the tile
+          uint8_t* row = smem + L::kStgOff + (cn >> 6) * L::kHChunk + rc * 128;
+          uint32_t cw[8];
           uint32_t sbw = 0;
 #pragma unroll
-          for (int g = 0; g < 2; ++g) {
+          for (int g = 0; g < 4; ++g) {
+            uint4* p0 = reinterpret_cast<uint4*>(row + (((2 * g) ^ (rc & 7)) << 4));
+            uint4* p1 = reinterpret_cast<uint4*>(row + (((2 * g + 1) ^ (rc & 7)) << 4));
+            const uint4 u0 = *p0, u1 = *p1;
+            const uint32_t yw[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+            uint32_t hw[8];
             float v[16];
 #pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              hw[e] = pack_bf16x2(gelu(__uint_as_float(yw[e] << 16)), gelu(__uint_as_float(yw[e] & 0xFFFF0000u)));
+              v[2 * e] = __uint_as_float(hw[e] << 16);
+              v[2 * e + 1] = __uint_as_float(hw[e] & 0xFFFF0000u);
+            }
+            *p0 = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            *p1 = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+            const float* is = is_tile + cn + 16 * g;
+#pragma unroll
             for (int e = 0; e < 16; e += 4) {
-              const float4 s4 = *reinterpret_cast<const float4*>(is + 16 * g + e);
-              const float2 a = __fmul2_rn(make_float2(hv[16 * g + e], hv[16 * g + e + 1]), make_float2(s4.x, s4.y));
-              const float2 b2 =
-                  __fmul2_rn(make_float2(hv[16 * g + e + 2], hv[16 * g + e + 3]), make_float2(s4.z, s4.w));
+              const float4 s4 = *reinterpret_cast<const float4*>(is + e);
+              const float2 a = __fmul2_rn(make_float2(v[e], v[e + 1]), make_float2(s4.x, s4.y));
+              const float2 b2 = __fmul2_rn(make_float2(v[e + 2], v[e + 3]), make_float2(s4.z, s4.w));
               v[e] = a.x;
               v[e + 1] = a.y;
               v[e + 2] = b2.x;
               v[e + 3] = b2.y;
             }
-            const uint32_t sb = nvfp4_quant16(v, mlp.denom, mlp.g_x, cw[2 * g], cw[2 * g + 1]);
-            sbw |= sb << (8 * g);
+            sbw |= nvfp4_quant16(v, mlp.denom, mlp.g_x, cw[2 * g], cw[2 * g + 1]) << (8 * g);
           }
           if (m < mlp.M_pad) {
-            *reinterpret_cast<uint4*>(mlp.codes + static_cast<size_t>(m) * (mlp.K >> 1) + (n >> 1)) =
-                make_uint4(cw[0], cw[1], cw[2], cw[3]);
-            // scale-factor atom (m / 128) * (K / 64) + n / 64; the chunk's two groups are adjacent bytes
+            const int n = nb * kBN + cn;  // column of the up output = k of the down layer
+            uint4* dst = reinterpret_cast<uint4*>(mlp.codes + static_cast<size_t>(m) * (mlp.K >> 1) + (n >> 1));
+            dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+            // scale-factor atom (m / 128) * (K / 64) + n / 64 holds the four groups as adjacent bytes
             const size_t atom = static_cast<size_t>(m >> 7) * (mlp.K >> 6) + (n >> 6);
-            const int off = (m & 31) * 16 + ((m >> 5) & 3) * 4 + ((n >> 4) & 3);
-            *reinterpret_cast<uint16_t*>(mlp.scales + atom * 512 + off) = static_cast<uint16_t>(sbw);
-          }
-          // stage h for the T contraction: K-major 128 x 64 chunks, 128-byte swizzle
-          uint8_t* hrow = smem + L::kStgOff + (cn >> 6) * L::kHChunk + rc * 128;
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const int chunk = ((cn & 63) >> 3) + v;
-            *reinterpret_cast<uint4*>(hrow + ((chunk ^ (rc & 7)) << 4)) =
-                make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+            *reinterpret_cast<uint32_t*>(mlp.scales + atom * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4) = sbw;
           }
         }
-      }
-      tc_fence_before();
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_cluster(acc_empty, 0);  // this CTA's share of TMEM is free
-        mbar_arrive(&bias_empty[bs]);
-        if (kMlp) {
+        fence_proxy_async_smem();  // h is read by the T contraction's MMAs
+        __syncwarp();
+        if (lane == 0) {
           mbar_arrive(&is_empty[bs]);
           mbar_arrive_cluster(h_ready, 0);
-        } else {
-#pragma unroll
-          for (int b = 0; b < 2; ++b) tma_store_2d(&maps.y, stg + b * L::kStgBox, nb * kBN + col0 + 64 * b, row0);
-          bulk_commit_group();
         }
       }
       // MLP: the previous tile closed a row block: its partial is complete (its
@@ -601,28 +649,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
 }
 
-// T = bf16(t_scale * sum over the partial slots of each 256-row block, in slot order).
+// T = bf16(t_scale * sum over the partial slots of each 256-row block, in slot
+// order); one thread per element, 8 rows per CTA.
+constexpr int kReduceRows = 8;
 __global__ void mlp_t_reduce_kernel(const float* tpart, int M_pad, int slots, int n_tiles, int n_blocks, int n_pairs,
                                     float t_scale, __nv_bfloat16* T) {
-  const int mp = blockIdx.x;
-  const int t0 = mp * n_blocks, t1 = t0 + n_blocks;  // the block's tiles
-  const int p0 = mlp_first_pair(mp, n_blocks, n_tiles, n_pairs);
-  int used = 0;  // pairs whose range holds a tile of this block
-  for (int pp = p0; pp < n_pairs; ++pp) {
-    const long long f = (static_cast<long long>(pp) * n_tiles) / n_pairs;
-    const long long l = (static_cast<long long>(pp + 1) * n_tiles) / n_pairs;
-    if (f >= t1) break;
-    if (l > t0 && l > f) ++used;
-  }
-  for (int i = threadIdx.x; i < 2 * kBM * kMlpDownRP; i += blockDim.x) {
-    const int r = i / kMlpDownRP, c = i % kMlpDownRP;
-    const int m = mp * 2 * kBM + r;
-    if (m >= M_pad) continue;
-    float acc = 0.f;
-    for (int sl = 0; sl < used && sl < slots; ++sl)
-      acc += tpart[((static_cast<size_t>(mp) * slots + sl) * (2 * kBM) + r) * kMlpDownRP + c];
-    T[static_cast<size_t>(m) * kMlpDownRP + c] = __float2bfloat16_rn(acc * t_scale);
-  }
+  const int mp = blockIdx.x / (2 * kBM / kReduceRows);
+  const int r = (blockIdx.x % (2 * kBM / kReduceRows)) * kReduceRows + threadIdx.x / kMlpDownRP;
+  const int c = threadIdx.x % kMlpDownRP;
+  const int m = mp * 2 * kBM + r;
+  __shared__ int used_s;  // pairs whose range holds a tile of this block
+  if (threadIdx.x == 0) used_s = mlp_block_pairs(mp, n_blocks, n_tiles, n_pairs);
+  __syncthreads();
+  const int used = used_s;
+  if (m >= M_pad) return;
+  const float* src = tpart + (static_cast<size_t>(mp) * slots * (2 * kBM) + r) * kMlpDownRP + c;
+  float acc = 0.f;
+  for (int sl = 0; sl < used && sl < slots; ++sl) acc += src[static_cast<size_t>(sl) * (2 * kBM) * kMlpDownRP];
+  T[static_cast<size_t>(m) * kMlpDownRP + c] = __float2bfloat16_rn(acc * t_scale);
 }
 
 int max_pairs_on_device() {
@@ -677,16 +721,8 @@ int nvfp4_pairs(int tiles) {
 
 int nvfp4_mlp_slots(int tiles, int n_blocks, int pairs) {
   int slots = 1;
-  const int m_blocks = tiles / n_blocks;
-  for (int mp = 0; mp < m_blocks; ++mp) {
-    const long long t0 = static_cast<long long>(mp) * n_blocks, t1 = t0 + n_blocks;
-    int used = 0;
-    for (int pp = mlp_first_pair(mp, n_blocks, tiles, pairs); pp < pairs; ++pp) {
-      const long long f = (static_cast<long long>(pp) * tiles) / pairs;
-      const long long l = (static_cast<long long>(pp + 1) * tiles) / pairs;
-      if (f >= t1) break;
-      if (l > t0 && l > f) ++used;
-    }
+  for (int mp = 0; mp < tiles / n_blocks; ++mp) {
+    const int used = mlp_block_pairs(mp, n_blocks, tiles, pairs);
     slots = used > slots ? used : slots;
   }
   return slots;
@@ -706,7 +742,7 @@ cudaError_t launch_gemm_nvfp4_mlp(const GemmParams& p, const MlpDownParams& mlp,
 cudaError_t launch_mlp_t_reduce(const float* tpart, int M_pad, int slots, int tiles, int n_blocks, int pairs,
                                 float t_scale, __nv_bfloat16* T, cudaStream_t stream) {
   const int m_blocks = (M_pad + 255) / 256;
-  mlp_t_reduce_kernel<<<m_blocks, 256, 0, stream>>>(tpart, M_pad, slots, tiles, n_blocks, pairs, t_scale, T);
+  mlp_t_reduce_kernel<<<m_blocks * (2 * kBM / kReduceRows), kReduceRows * kMlpDownRP, 0, stream>>>(tpart, M_pad, slots, tiles, n_blocks, pairs, t_scale, T);
   return cudaGetLastError();
 }
 

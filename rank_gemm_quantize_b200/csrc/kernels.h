@@ -26,6 +26,7 @@ struct ActQuantParams {
   uint8_t* codes;          // INT4: [M_pad, K] E4M3 bytes of the integer codes; NVFP4: [M_pad, K/2] packed E2M1
   void* scales;            // INT4: float [K/64][M_pad]; NVFP4: scale-factor atoms [M_pad/128][K/64][512]
   __nv_bfloat16* T;        // [M_pad, RP] bf16 = t_scale * (x_hat L1)
+  __nv_bfloat16* T_lo;     // NULL, or [M_pad, RP]: bf16(v - T) of the same float v (T + T_lo ~ 16 bits of v)
   int split;               // K shares per 128-row block (from act_quant_split)
   float* Tpart;            // [split][M_pad][RP] float partials over the K shares (split > 1)
   int* counters;           // [M_pad / 128] arrival counts of the shares, zero between launches
@@ -76,6 +77,7 @@ struct GemmMaps {
   CUtensorMap y;    // NVFP4: Y [M, N] bf16, box {64, 32}, 128-byte swizzle (TMA stores)
   CUtensorMap l1h_down;  // MLP block: the down layer's L1s^T high part [RP_down, K_down], box {64, RP_down / 2}
   CUtensorMap l1l_down;  // ... and low part
+  CUtensorMap t_lo;      // MLP block: the up layer's T low part [M_pad, RP] bf16, as t
 };
 
 // The down layer of an MLP block as the fused epilogue of the up layer's

@@ -83,7 +83,8 @@ struct MapCache {
   struct Entry {
     const void* key = nullptr;
     int rows = -1;
-    CUtensorMap a{}, b{}, c{};
+    CUtensorMap a{}, b{}, c{}, d{};
+    const void* dkey = nullptr;  // the buffer map d was made for (built on first use)
   };
   Entry e[N];
   int next = 0;
@@ -559,7 +560,8 @@ svdq_status svd_factors(svdq_layer* h, const float* W_hat, __nv_bfloat16* L1, __
 }
 
 svdq_status launch_k1(svdq_layer* h, const void* X, int M, uint8_t* codes, void* scales, __nv_bfloat16* T,
-                      float* Tpart, const WsLayout& w, const uint32_t* row_mask, cudaStream_t st) {
+                      float* Tpart, const WsLayout& w, const uint32_t* row_mask, cudaStream_t st,
+                      __nv_bfloat16* T_lo = nullptr) {
   if (w.M_pad / 128 > kMaxRowBlocks) return fail(SVDQ_ERR_INVALID_ARG, "M exceeds the supported row count");
   ActQuantParams p{};
   p.split = w.split;
@@ -573,6 +575,7 @@ svdq_status launch_k1(svdq_layer* h, const void* X, int M, uint8_t* codes, void*
   p.codes = codes;
   p.scales = scales;
   p.T = T;
+  p.T_lo = T_lo;
   p.g_x = h->g_x;
   p.denom = h->denom;
   p.t_scale = h->t_scale;
@@ -699,7 +702,7 @@ namespace {
 // layer of an MLP block: its epilogue writes the down layer's activations
 // instead of Y.
 svdq_status gemm_stage(svdq_layer* h, int M, void* Y, uint8_t* codes, void* scales, __nv_bfloat16* T,
-                       const MlpDownParams* mlp, const GemmMaps* mlp_maps, cudaStream_t st) {
+                       __nv_bfloat16* T_lo, const MlpDownParams* mlp, const GemmMaps* mlp_maps, cudaStream_t st) {
   const int M_pad = round_up(M, 128);
   auto* we = h->ws_maps.find(codes, M);
   if (!we) {
@@ -708,6 +711,8 @@ svdq_status gemm_stage(svdq_layer* h, int M, void* Y, uint8_t* codes, void* scal
     const uint64_t row = i4 ? h->K : h->K / 2;
     we->b = CUtensorMap{};
     we->c = CUtensorMap{};
+    we->d = CUtensorMap{};
+    we->dkey = nullptr;
     if (!make_map(&we->a, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, row, M_pad, row, 128, kActBoxRows,
                   CU_TENSOR_MAP_SWIZZLE_128B) ||
         (!i4 && !make_sf_map(&we->c, scales, static_cast<uint64_t>(M_pad / 128) * (h->K / 64))) ||
@@ -716,6 +721,14 @@ svdq_status gemm_stage(svdq_layer* h, int M, void* Y, uint8_t* codes, void* scal
       we->key = nullptr;
       return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (activations) failed");
     }
+  }
+  if (h->RP > 0 && T_lo && we->dkey != T_lo) {  // the MLP block's T low part
+    if (!make_map(&we->d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, T_lo, h->RP, M_pad, static_cast<uint64_t>(h->RP) * 2, 32,
+                  128, CU_TENSOR_MAP_SWIZZLE_64B)) {
+      we->key = nullptr;
+      return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (T low part) failed");
+    }
+    we->dkey = T_lo;
   }
   GemmParams p{};
   p.M = M;
@@ -737,6 +750,7 @@ svdq_status gemm_stage(svdq_layer* h, int M, void* Y, uint8_t* codes, void* scal
   maps.l2 = h->map_l2;
   maps.sfa = we->c;
   maps.sfb = h->map_sfb;
+  maps.t_lo = we->d;
   if (h->fmt == SVDQ_NVFP4_G16 && !mlp) {
     auto* ye = h->y_maps.find(Y, M);
     if (!ye) {
@@ -779,7 +793,7 @@ svdq_status forward_impl(svdq_layer* h, const void* X, int M, void* Y, void* wor
   svdq_status e = launch_k1(h, X, M, codes, scales, T, Tpart, w, row_mask, st);
   if (e) return e;
   if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[1]), st));
-  if ((e = gemm_stage(h, M, Y, codes, scales, T, nullptr, nullptr, st))) return e;
+  if ((e = gemm_stage(h, M, Y, codes, scales, T, nullptr, nullptr, nullptr, st))) return e;
   if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[2]), st));
   return SVDQ_OK;
 }
@@ -788,7 +802,7 @@ svdq_status forward_impl(svdq_layer* h, const void* X, int M, void* Y, void* wor
 // down layer's activation codes, scales and T, and the T partials.
 struct MlpLayout {
   WsLayout up, down;
-  size_t down_off, tpart_off, total;
+  size_t down_off, tpart_off, tlo_off, total;
   int tiles, n_blocks, pairs, slots;
 };
 
@@ -803,7 +817,8 @@ MlpLayout mlp_layout(const svdq_layer* up, const svdq_layer* down, int M) {
   l.pairs = nvfp4_pairs(l.tiles);
   l.slots = nvfp4_mlp_slots(l.tiles, l.n_blocks, l.pairs);
   const size_t tpart = static_cast<size_t>((l.up.M_pad + 255) / 256) * l.slots * 256 * kMlpDownRP * 4;
-  l.total = l.tpart_off + align256(tpart);
+  l.tlo_off = l.tpart_off + align256(tpart);  // the up layer's T low part
+  l.total = l.tlo_off + align256(static_cast<size_t>(l.up.M_pad) * up->RP * 2);
   return l;
 }
 
@@ -835,6 +850,7 @@ svdq_status mlp_impl(svdq_layer* up, svdq_layer* down, const void* X, int M, voi
   uint8_t* scales_d = dbase + l.down.scales;
   __nv_bfloat16* T_d = reinterpret_cast<__nv_bfloat16*>(dbase + l.down.T);
   float* tpart = reinterpret_cast<float*>(base + l.tpart_off);
+  __nv_bfloat16* T_lo = up->RP > 0 ? reinterpret_cast<__nv_bfloat16*>(base + l.tlo_off) : nullptr;
   // the down layer's factor as the fused epilogue loads it: each CTA of a pair its 16 rows
   if (!down->mlp_maps_ready) {
     if (!make_map(&down->map_l1h_half, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, down->L1sTh, down->K, down->RP,
@@ -847,7 +863,7 @@ svdq_status mlp_impl(svdq_layer* up, svdq_layer* down, const void* X, int M, voi
   if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[0]), st));
   svdq_status e = launch_k1(up, X, M, base + l.up.codes, base + l.up.scales,
                             reinterpret_cast<__nv_bfloat16*>(base + l.up.T), reinterpret_cast<float*>(base + l.up.Tpart),
-                            l.up, nullptr, st);
+                            l.up, nullptr, st, T_lo);
   if (e) return e;
   if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[1]), st));
   MlpDownParams mp{};
@@ -864,13 +880,13 @@ svdq_status mlp_impl(svdq_layer* up, svdq_layer* down, const void* X, int M, voi
   extra.l1h_down = down->map_l1h_half;
   extra.l1l_down = down->map_l1l_half;
   if ((e = gemm_stage(up, M, nullptr, base + l.up.codes, base + l.up.scales,
-                      reinterpret_cast<__nv_bfloat16*>(base + l.up.T), &mp, &extra, st)))
+                      reinterpret_cast<__nv_bfloat16*>(base + l.up.T), T_lo, &mp, &extra, st)))
     return e;
   if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[2]), st));
   cudaError_t ce = launch_mlp_t_reduce(tpart, l.down.M_pad, l.slots, l.tiles, l.n_blocks, l.pairs, down->t_scale, T_d, st);
   if (ce != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("T reduction: ") + cudaGetErrorString(ce));
   if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[3]), st));
-  if ((e = gemm_stage(down, M, Y, codes_d, scales_d, T_d, nullptr, nullptr, st))) return e;
+  if ((e = gemm_stage(down, M, Y, codes_d, scales_d, T_d, nullptr, nullptr, nullptr, st))) return e;
   if (events) CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[4]), st));
   return SVDQ_OK;
 }

@@ -7,15 +7,19 @@ block's two layers). The oracle runs the plain composition: the up layer in
 float64, its output rounded to bf16, exact-erf GELU rounded to bf16, the
 down layer.
 
-The two sides compute the up layer's output in different precisions (float32
-tensor-core accumulation vs float64) and GELU with different erf routines, so
-h = bf16(GELU(bf16(y))) can legitimately differ by one bf16 unit where a value
-sits on a rounding boundary. The down layer's codes and scales are therefore
-compared bit for bit on every quantization group whose sixteen h values are
-decided: the oracle's float64 y lies farther than a margin from a bf16
-rounding boundary, and so does its exact GELU value. Every other group is
-checked for validity (scale within one E4M3 step, codes within one E2M1
-step). T and Y are compared within the usual 2e-3 / 4e-3 normwise bounds.
+The two sides reach h = bf16(GELU(bf16(y))) along different roundings: the
+kernel accumulates in float32, carries the up layer's branch input T as a
+bf16 pair (T + T_lo, about 16 significant bits) and evaluates erf in float32.
+Where y or GELU(y) lies close to a bf16 rounding boundary, h may
+legitimately come out one bf16 step apart. So the down layer's codes and
+scales are checked against intervals: a bound on the kernel's deviation in y
+(from the sums of absolute terms of each product) gives, per element, the
+bf16 values y and then h can take; through the smoothing and the group
+maximum that gives the range of valid E4M3 scales of each group, and, given
+the kernel's scale, the range of valid E2M1 codes of each element. Where the
+range holds one value (almost every group and element) the comparison is
+exact, bit for bit; elsewhere the kernel's value must lie inside it. T and Y
+are compared within the single layer's 2e-3 / 4e-3 normwise bounds.
 """
 import numpy as np
 import pytest
@@ -28,19 +32,77 @@ from parity import T_TOL, Y_TOL, bf16_tensor, f64, rel
 
 pytestmark = pytest.mark.gpu
 
-Y_MARGIN = 2e-5    # relative: float32 accumulation of the up GEMM against float64
-G_MARGIN = 2e-6    # relative: float32 erf-GELU against the exact one
+F32 = np.float32
+GELU_ARGMIN = -0.7517915246935645  # GELU is decreasing left of this point, increasing right of it
+# |GELU_kernel(y) - GELU(y)| <= E_GELU_Y |y| + E_GELU_G |GELU(y)|: the kernel's erf is within
+# about 5e-7 of the exact one (absolute), then float32 products
+E_GELU_Y = 1e-6
+E_GELU_G = 2.0 ** -21
 
 
-def _far_from_bf16_boundary(x, margin):
-    """|x| is farther than margin * |x| from the midpoint between its two
-    neighbouring bf16 values (so any estimate within that margin rounds alike)."""
-    x = np.asarray(x, dtype=np.float64)
-    _, e = np.frexp(x)
-    ulp = np.ldexp(1.0, np.maximum(e - 8, -133))
-    frac = np.abs(x) / ulp - np.floor(np.abs(x) / ulp)
-    dist = np.abs(frac - 0.5) * ulp
-    return dist > margin * np.abs(x) + 1e-30
+def _up_output_bound(p, X, fr):
+    """Per element, a bound on |y_kernel - y_oracle| for the up layer's output
+    before its bf16 rounding: T as a float32 accumulation over K held as a
+    bf16 pair (2^-16 relative), float32 accumulation of the 4-bit and branch
+    products, the tensor-scale product and the bias; each term with a factor
+    of at least 2 to spare."""
+    x_hat = S.smooth_activations(X, p.inv_s).astype(np.float64)
+    xq = F.dequantize(fr.x_codes, fr.x_scales, p.fmt, p.g_x)
+    wq = S.dequantized_weight(p)
+    absT = np.abs(fr.T)
+    e_T = 2.0 ** -15 * (absT + np.abs(x_hat) @ np.abs(p.L1))
+    return (e_T @ np.abs(p.L2)
+            + 2.0 ** -15 * (np.abs(xq) @ np.abs(wq).T + absT @ np.abs(p.L2))
+            + 2.0 ** -20 * (np.abs(fr.Y) + np.abs(p.bias)[None, :]))
+
+
+def _h_interval(y, e_y):
+    """The bf16 values h = bf16(GELU(bf16(y'))) can take for |y' - y| <= e_y
+    and a kernel GELU within the stated error: [h_lo, h_hi]."""
+    y_lo, y_hi = F.bf16_round(y - e_y), F.bf16_round(y + e_y)
+    g_a, g_b = S.gelu_erf(y_lo), S.gelu_erf(y_hi)
+    g_min = np.minimum(g_a, g_b)
+    inside = (y_lo < GELU_ARGMIN) & (y_hi > GELU_ARGMIN)
+    g_min = np.where(inside, np.minimum(g_min, S.gelu_erf(np.float64(GELU_ARGMIN))), g_min)
+    g_max = np.maximum(g_a, g_b)
+    e_g = E_GELU_Y * np.maximum(np.abs(y_lo), np.abs(y_hi)) + E_GELU_G * np.maximum(np.abs(g_a), np.abs(g_b))
+    return F.bf16_round(g_min - e_g), F.bf16_round(g_max + e_g)
+
+
+def _check_down_quantization(h_lo, h_hi, p_dn, q_gpu, sc_gpu, q_ref, sc_ref):
+    """The kernel's scales and codes of the down layer lie in the ranges that
+    [h_lo, h_hi] allows; exact where a range holds one value. Returns the
+    decided fractions (scales, codes)."""
+    R = h_lo.shape[0]
+    inv = np.asarray(p_dn.inv_s, dtype=F32)[None, :]
+    x_lo = (h_lo.astype(F32) * inv).astype(F32).reshape(R, -1, 16)
+    x_hi = (h_hi.astype(F32) * inv).astype(F32).reshape(R, -1, 16)
+    straddle = (x_lo <= 0) & (x_hi >= 0)
+    a_lo = np.where(straddle, F32(0), np.minimum(np.abs(x_lo), np.abs(x_hi))).max(axis=-1)
+    a_hi = np.maximum(np.abs(x_lo), np.abs(x_hi)).max(axis=-1)
+    g = F32(p_dn.g_x)
+    denom = F32(F32(6.0) * g)
+    sb_lo = F.e4m3_encode((a_lo.astype(F32) / denom).astype(F32)).astype(int)
+    sb_hi = F.e4m3_encode((a_hi.astype(F32) / denom).astype(F32)).astype(int)
+    assert np.all((sb_lo <= sc_ref) & (sc_ref <= sb_hi)), "the oracle's own scales fall outside the ranges"
+    sc = sc_gpu.astype(int)
+    bad = ~((sb_lo <= sc) & (sc <= sb_hi))
+    assert not bad.any(), f"{bad.sum()} of {bad.size} group scales outside their valid range"
+    one = sb_lo == sb_hi
+    assert np.array_equal(sc[one], sc_ref[one].astype(int))
+    # codes, given the kernel's scale of each group
+    eff = (F.e4m3_decode(sc_gpu).astype(F32) * g).astype(F32)
+    zero = eff == 0
+    inv_e = (F32(1.0) / np.where(zero, F32(1), eff)).astype(F32)[..., None]
+    c_lo = np.where(zero[..., None], 0, F.e2m1_encode((x_lo * inv_e).astype(F32)))
+    c_hi = np.where(zero[..., None], 0, F.e2m1_encode((x_hi * inv_e).astype(F32)))
+    v_lo, v_hi, v = F.e2m1_decode(c_lo), F.e2m1_decode(c_hi), F.e2m1_decode(q_gpu)
+    bad = ~((v_lo <= v) & (v <= v_hi))
+    assert not bad.any(), f"{bad.sum()} of {bad.size} codes outside their valid range"
+    c_one = (c_lo == c_hi) & one[..., None]
+    assert np.array_equal(q_gpu[c_one], c_lo[c_one].astype(q_gpu.dtype))
+    assert np.array_equal(q_gpu[c_one], q_ref[c_one])  # there the oracle's code is the only valid one
+    return one.mean(), c_one.mean()
 
 
 def _block(M, K, N, Kd_out, seed):
@@ -85,29 +147,25 @@ def _run(up, Wd, bd, rows=None):
         g_dn.close()
     r = np.arange(up.M) if rows is None else rows
     res = S.mlp_forward(p_up, p_dn, X[r])
-    # y_up of the oracle before rounding, for the decidability margin
-    y_exact = S.forward(p_up, X[r]).Y
-    decided_y = _far_from_bf16_boundary(y_exact, Y_MARGIN)
-    decided_g = _far_from_bf16_boundary(S.gelu_erf(res.y_up), G_MARGIN)
-    decided = (decided_y & decided_g).reshape(len(r), -1, 16).all(axis=-1)  # per group of 16
+    fr_up = S.forward(p_up, X[r])
+    h_lo, h_hi = _h_interval(fr_up.Y, _up_output_bound(p_up, X[r], fr_up))
+    assert np.all((h_lo <= res.h) & (res.h <= h_hi))
     q = F.unpack_nibbles(codes[r], signed=False)
     m = np.asarray(r)[:, None]
     i = np.arange(Kd // 16)[None, :]
     sc = atoms[((m // 128) * (Kd // 64) + i // 4) * 512 + (m % 32) * 16 + ((m // 32) % 4) * 4 + i % 4]
-    want_q, want_s = res.down.x_codes, res.down.x_scales
     qg = q.reshape(len(r), -1, 16)
-    wg = want_q.reshape(len(r), -1, 16)
-    assert decided.mean() > 0.9, decided.mean()
-    assert np.array_equal(sc[decided], want_s[decided])
-    assert np.array_equal(qg[decided], wg[decided])
-    # undecided groups: valid neighbours of the oracle's result
-    und = ~decided
-    assert np.all(np.abs(sc[und].astype(int) - want_s[und].astype(int)) <= 1)
-    mag = lambda c: F.e2m1_decode(c)
-    assert np.all(np.abs(mag(qg[und]) - mag(wg[und])) <= 2.0 + 1e-12)  # adjacent E2M1 values (or a scale step)
+    wg = res.down.x_codes.reshape(len(r), -1, 16)
+    s_one, c_one = _check_down_quantization(h_lo, h_hi, p_dn, qg, sc, wg, res.down.x_scales)
+    # the bound is worst-case, so the exact comparison covers most but not all of the tensor
+    # (scales 99-99.5 %, codes 91-97 % on the small shapes and 73 % on the FLUX block) ...
+    assert s_one > 0.95 and c_one > 0.6, (s_one, c_one)
+    # ... while the kernel's typical deviation is far smaller: nearly every scale and code is the
+    # oracle's own (over 99.99 % when T is a bf16 pair and everything else is exact)
+    assert (sc == res.down.x_scales).mean() > 0.995 and (qg == wg).mean() > 0.995
     assert rel(T[r], res.down.T) <= T_TOL
     assert rel(y[r], res.down.Y) <= Y_TOL
-    return decided.mean()
+    return s_one, c_one
 
 
 @pytest.mark.parametrize("M,K,N,Kd_out,seed", [(200, 512, 512, 256, 121), (384, 256, 1024, 512, 122)])
