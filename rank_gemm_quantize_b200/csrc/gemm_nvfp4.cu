@@ -20,21 +20,23 @@
 // of the pair read both CTAs' halves. Per SM that is 38 KB of operands per
 // 256-deep k-tile instead of 54 KB for a 128 x 256 tile on one SM.
 //
-// Persistent kernel, one pair per two SMs. Warp roles (11 warps per CTA):
+// Persistent kernel, one pair per two SMs. Warp roles (19 warps per CTA):
 //   warp 0  producer (both CTAs): per tile its bias slice (bulk copy, local
 //           ring), then the k-tiles: A and B codes and both scale-factor
 //           tiles by TMA, completing on the leader CTA's stage barrier;
 //           then the branch k-tiles (32-column slices of T' and L2^T);
-//   warp 10 scale factors (leader): copies each stage's scale factors of both
+//   warp 18 scale factors (leader): copies each stage's scale factors of both
 //           CTAs into their TMEM (tcgen05.cp .cta_group::2) and commits;
 //   warp 1  TMEM owner (both) and MMA issuer (leader, one thread): per k-tile
 //           4 block-scaled MMAs, per branch k-tile 2 kind::f16 MMAs; the
 //           commits free the stage in both CTAs and mark the tile;
-//   warps 2-9 epilogue (both): each reads its 32 rows x 128 columns of its
+//   warps 2-17 epilogue (both), four per TMEM lane quarter (enough warps to
+//           hide the latency of the MLP variant's per-element work): each
+//           reads its 32 rows x 64 columns of its
 //           CTA's accumulator 32 columns at a time, scales, adds the bias,
 //           packs bf16 and writes it into a 128-byte-swizzled staging buffer
 //           right away; then it tells the leader that TMEM is free (the next
-//           tile's MMAs start) and stores its two 32 x 64 boxes with TMA
+//           tile's MMAs start) and stores its 32 x 64 box with TMA
 //           (rows and columns past M and N are clipped by the tensor map).
 //
 // MLP-block variant (kMlp, the up layer of up -> GELU -> down): the branch
@@ -66,7 +68,8 @@ constexpr int kBM = 128;       // rows per CTA (the pair covers 256)
 constexpr int kBN = 256;       // columns per pair tile
 constexpr int kBNHalf = 128;   // weight rows each CTA loads
 constexpr int kBKBytes = 128;  // 256 E2M1 values per row per k-tile
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;                   // four per TMEM lane quarter
+constexpr int kEpiCols = kBN / (kEpiWarps / 4);  // columns of the tile each epilogue warp takes (64)
 constexpr int kCpWarp = 2 + kEpiWarps;  // copies scale factors into TMEM
 constexpr int kThreads = (3 + kEpiWarps) * 32;
 
@@ -80,11 +83,11 @@ struct SmemNv {
   static constexpr int kStage = kA + kB + kSfa + kSfb;  // 38 KB
   static constexpr int kBiasOff = kStages * kStage;
   static constexpr int kBias = kBN * 2;           // bf16 bias slice of a tile
-  // Y staging for the TMA stores (8 warps x two 32 x 64 boxes); in the MLP
+  // Y staging for the TMA stores (16 warps x one 32 x 64 box); in the MLP
   // variant the same 64 KB hold h as four K-major 128 x 64 bf16 chunks.
   static constexpr int kStgOff = kBiasOff + 2 * kBias;
   static constexpr int kStgBox = 32 * 128;
-  static constexpr int kStgWarp = 2 * kStgBox;
+  static constexpr int kStgWarp = (kEpiCols / 64) * kStgBox;
   static constexpr int kStg = kEpiWarps * kStgWarp;  // 64 KB
   static constexpr int kHChunk = kBM * 128;          // 16 KB: 128 rows x 64 bf16
   static constexpr int kIsOff = kStgOff + kStg;      // MLP: down-layer inv_s slices, 2 x 256 floats
@@ -467,7 +470,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int ew = warp - 2;                  // 0..7
     const int q = warp & 3;                   // TMEM lane quarter this warp may access
-    const int col0 = (ew >> 2) * (kBN / 2);   // this warp's half of the tile's columns
+    const int col0 = (ew >> 2) * kEpiCols;    // this warp's columns of the tile
     const int rc = 32 * q + lane;             // this thread's row within the CTA's 128
     uint8_t* stg = smem + L::kStgOff + ew * L::kStgWarp;
     bool ok = true;
@@ -514,7 +517,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // Phase A: the accumulator -> y = out_scale acc + b, bf16, into the staging buffer (the Y
       // boxes; in the MLP block the K-major h chunks, where phase B turns y into h in place)
 #pragma unroll
-      for (int c = 0; c < kBN / 64; ++c) {  // 32 columns: half of one 64-column staging box
+      for (int c = 0; c < kEpiCols / 32; ++c) {  // 32 columns: half of one 64-column staging box
         uint32_t r[32];
         tmem_ld32(ta + 32 * c, r);
         tmem_ld_wait();
@@ -554,7 +557,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mbar_arrive(&bias_empty[bs]);
         if (!kMlp) {
 #pragma unroll
-          for (int b = 0; b < 2; ++b) tma_store_2d(&maps.y, stg + b * L::kStgBox, nb * kBN + col0 + 64 * b, row0);
+          for (int b = 0; b < kEpiCols / 64; ++b)
+            tma_store_2d(&maps.y, stg + b * L::kStgBox, nb * kBN + col0 + 64 * b, row0);
           bulk_commit_group();
         }
       }
@@ -564,7 +568,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const float* is_tile = reinterpret_cast<const float*>(smem + L::kIsOff + bs * L::kIs);
         const int m = row0 + lane;
 #pragma unroll 1
-        for (int piece = 0; piece < 2; ++piece) {
+        for (int piece = 0; piece < kEpiCols / 64; ++piece) {
           const int cn = col0 + 64 * piece;  // first column of the 64 within the tile
           uint8_t* row = smem + L::kStgOff + (cn >> 6) * L::kHChunk + rc * 128;
           uint32_t cw[8];
