@@ -202,7 +202,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint64_t* h_ready = l1_empty + 2;      // (leader) both CTAs staged the tile's h
   uint64_t* t_full = h_ready + 1;        // (both) T accumulator holds a finished row-block partial
   uint64_t* t_empty = t_full + 1;        // (leader) both CTAs read that partial out
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(t_empty + 1);
+  uint64_t* sf_full = t_empty + 1;       // [kStages] (leader) both CTAs' scale-factor tiles of the stage landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_full + kStages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -225,6 +226,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&sf_ready[s], 1);
+      mbar_init(&sf_full[s], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * kEpiWarps);
@@ -295,18 +297,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           uint8_t* st = smem + s * L::kStage;
           const uint32_t fb = leader_addr(&full[s]);
           if (k < n_main) {
-            if (leader) mbar_arrive_expect_tx(&full[s], 2 * L::kStage);
+            // the scale factors first, on their own barrier: their copies into TMEM overlap the
+            // landing of the codes instead of following it
+            const uint32_t sb = leader_addr(&sf_full[s]);
+            if (leader) {
+              mbar_arrive_expect_tx(&sf_full[s], 2 * (L::kSfa + L::kSfb));
+              mbar_arrive_expect_tx(&full[s], 2 * (L::kA + L::kB));
+            }
             const int kb0 = k * 4;
-            tma_load_2d_pair(st, &maps.a, fb, k * kBKBytes, m0);
-            tma_load_2d_pair(st + L::kA, &maps.b, fb, k * kBKBytes, n0 + static_cast<int>(rank) * kBNHalf);
             // scale-factor atoms (512 bytes each): 4 k-blocks of this CTA's row block, and of both column blocks
-            tma_load_2d_pair(st + L::kA + L::kB, &maps.sfa, fb, 0, (m0 / 128) * kb_total + kb0);
+            tma_load_2d_pair(st + L::kA + L::kB, &maps.sfa, sb, 0, (m0 / 128) * kb_total + kb0);
 #pragma unroll
             for (int h = 0; h < kBN / 128; ++h)
-              tma_load_2d_pair(st + L::kA + L::kB + L::kSfa + h * 2048, &maps.sfb, fb, 0,
+              tma_load_2d_pair(st + L::kA + L::kB + L::kSfa + h * 2048, &maps.sfb, sb, 0,
                                (nb * (kBN / 128) + h) * kb_total + kb0);
+            tma_load_2d_pair(st, &maps.a, fb, k * kBKBytes, m0);
+            tma_load_2d_pair(st + L::kA, &maps.b, fb, k * kBKBytes, n0 + static_cast<int>(rank) * kBNHalf);
           } else {
-            if (leader) mbar_arrive_expect_tx(&full[s], 2 * ((kMlp ? 2 : 1) * kBM * 64 + kBNHalf * 64));
+            if (leader) {
+              mbar_arrive(&sf_full[s]);  // no scale factors in a branch k-tile
+              mbar_arrive_expect_tx(&full[s], 2 * ((kMlp ? 2 : 1) * kBM * 64 + kBNHalf * 64));
+            }
             const int c = k - n_main;  // 32-column slice of the branch
             tma_load_2d_pair(st, &maps.t, fb, c * 32, m0);
             if (kMlp) tma_load_2d_pair(st + kBM * 64, &maps.t_lo, fb, c * 32, m0);
@@ -388,7 +399,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_after();
         for (int k = 0; k < n_items && ok; ++k, ++it) {
           const int s = it % kStages;
-          ok = mbar_wait(&sf_ready[s], (it / kStages) & 1, abort_flag, p.status);
+          ok = mbar_wait(&full[s], (it / kStages) & 1, abort_flag, p.status) &&
+               mbar_wait(&sf_ready[s], (it / kStages) & 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
           if (lane == 0) {  // one fixed thread issues every tcgen05 op, so its commits track them all
@@ -440,7 +452,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int tile = tr.first; tile < tr.last && ok; tile += tr.step) {
         for (int k = 0; k < n_items && ok; ++k, ++it) {
           const int s = it % kStages;
-          ok = mbar_wait(&full[s], (it / kStages) & 1, abort_flag, p.status);
+          ok = mbar_wait(&sf_full[s], (it / kStages) & 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
           if (k < n_main) {
