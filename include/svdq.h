@@ -171,8 +171,9 @@ SVDQ_API svdq_status svdq_linear_forward_profiled(svdq_layer_t layer, const void
 
 /* The MLP block of two layers, Y = down(GELU(up(X))), fused across the
  * boundary between them: the up layer's GEMM epilogue rounds its output to
- * bf16, applies GELU (the erf form in float32, erf by Abramowitz & Stegun
- * 7.1.26, absolute error under 1e-6) and rounds to bf16 (h, what a plain
+ * bf16, applies GELU (the erf form in float32, erfc as exp(-x^2) times a
+ * fitted polynomial for erfcx, absolute error under 1e-6) and rounds to bf16
+ * (h, what a plain
  * composition of the layers would pass on), then smooths and quantizes
  * h for the down layer straight into the down layer's activation codes and
  * scales, and contracts it with the down layer's factor for the down layer's

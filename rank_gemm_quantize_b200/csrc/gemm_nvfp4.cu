@@ -122,22 +122,47 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// GELU(y) = y Phi(y) = 0.5 y (1 + erf(y / sqrt 2)), with erf by the rational
-// approximation of Abramowitz and Stegun, Handbook of Mathematical Functions,
-// formula 7.1.26: for x >= 0, erfc(x) ~ t (a1 + t (a2 + t (a3 + t (a4 + t a5))))
-// exp(-x^2), t = 1 / (1 + p x), absolute error at most 1.5e-7. The negative
-// side uses 1 + erf(-x) = erfc(x) directly, so no cancellation; with the
-// float32 evaluation the result is within about 5e-7 of 1 + erf, absolute.
-// The same instructions on every lane (no branch on the argument).
-__device__ __forceinline__ float gelu(float y) {
-  const float x = fabsf(y) * 0.70710678118654752f;
-  const float t = __fdividef(1.0f, fmaf(0.3275911f, x, 1.0f));
-  float poly = fmaf(1.061405429f, t, -1.453152027f);
-  poly = fmaf(poly, t, 1.421413741f);
-  poly = fmaf(poly, t, -0.284496736f);
-  poly = fmaf(poly, t, 0.254829592f);
-  const float erfc_x = poly * t * __expf(-x * x);
-  return 0.5f * y * (y >= 0.f ? 2.0f - erfc_x : erfc_x);
+// GELU(y) = y Phi(y) = y (1 + erf(y / sqrt 2)) / 2 of a packed bf16 pair,
+// returned as the packed bf16 pair of the results. With x = |y| / sqrt 2,
+// (1 + erf(y / sqrt 2)) / 2 is 1 - erfc(x) / 2 for y >= 0 and erfc(x) / 2 for
+// y < 0 (no cancellation on the negative side), and
+//   erfc(x) / 2 = 2^(-u^2) q(u),  u = |y| sqrt(log2(e) / 2),
+// where q(u) = erfcx(x) / 2 is approximated on [0, 6 sqrt(log2 e)] by a
+// degree-10 polynomial whose coefficients were fitted here by weighted
+// minimax (Lawson's iteration) with weight 2^(-u^2), so that the fit's error
+// is measured on erfc itself: at most 2.7e-7 absolute in float32 (u is
+// clamped at the end of that range, where erfc < 3e-17). Both values go
+// through packed float32 arithmetic (two per instruction); one ex2 each.
+__device__ __forceinline__ float ex2_approx(float v) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+  return r;
+}
+__device__ __forceinline__ uint32_t gelu_bf16x2(uint32_t w) {
+  const float2 y = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  const uint32_t a = w & 0x7FFF7FFFu;  // |y|
+  float2 u = __fmul2_rn(make_float2(__uint_as_float(a << 16), __uint_as_float(a & 0xFFFF0000u)),
+                        make_float2(8.493217826e-01f, 8.493217826e-01f));
+  u.x = fminf(u.x, 7.206734657e+00f);
+  u.y = fminf(u.y, 7.206734657e+00f);
+  const float2 uu = __fmul2_rn(u, u);
+  float2 q = make_float2(8.354404599e-06f, 8.354404599e-06f);
+  q = __ffma2_rn(q, u, make_float2(-1.531047310e-04f, -1.531047310e-04f));
+  q = __ffma2_rn(q, u, make_float2(1.254777540e-03f, 1.254777540e-03f));
+  q = __ffma2_rn(q, u, make_float2(-6.194117013e-03f, -6.194117013e-03f));
+  q = __ffma2_rn(q, u, make_float2(2.115210705e-02f, 2.115210705e-02f));
+  q = __ffma2_rn(q, u, make_float2(-5.501661450e-02f, -5.501661450e-02f));
+  q = __ffma2_rn(q, u, make_float2(1.175282001e-01f, 1.175282001e-01f));
+  q = __ffma2_rn(q, u, make_float2(-2.162939161e-01f, -2.162939161e-01f));
+  q = __ffma2_rn(q, u, make_float2(3.464582562e-01f, 3.464582562e-01f));
+  q = __ffma2_rn(q, u, make_float2(-4.697118402e-01f, -4.697118402e-01f));
+  q = __ffma2_rn(q, u, make_float2(4.999999404e-01f, 4.999999404e-01f));
+  const float2 hc = __fmul2_rn(make_float2(ex2_approx(-uu.x), ex2_approx(-uu.y)), q);  // erfc(x) / 2
+  // 1 - erfc/2 for y >= 0 (sign bit clear), erfc/2 itself for y < 0
+  const float2 om = __ffma2_rn(hc, make_float2(-1.f, -1.f), make_float2(1.f, 1.f));
+  const float2 t = make_float2((w & 0x8000u) ? hc.x : om.x, (w & 0x80000000u) ? hc.y : om.y);
+  const float2 g = __fmul2_rn(y, t);
+  return pack_bf16x2(g.x, g.y);
 }
 
 // The tile range of pair `pair`: round-robin for the plain GEMM (the pairs in
@@ -539,11 +564,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint4 bw = bias4[4 * c + v];
           const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            o[4 * v + e] =
-                pack_bf16x2(fmaf(__uint_as_float(r[8 * v + 2 * e]), p.out_scale, __uint_as_float(bb[e] << 16)),
-                            fmaf(__uint_as_float(r[8 * v + 2 * e + 1]), p.out_scale,
-                                 __uint_as_float(bb[e] & 0xFFFF0000u)));
+          for (int e = 0; e < 4; ++e) {
+            const float2 yv = __ffma2_rn(make_float2(__uint_as_float(r[8 * v + 2 * e]), __uint_as_float(r[8 * v + 2 * e + 1])),
+                                         make_float2(p.out_scale, p.out_scale),
+                                         make_float2(__uint_as_float(bb[e] << 16), __uint_as_float(bb[e] & 0xFFFF0000u)));
+            o[4 * v + e] = pack_bf16x2(yv.x, yv.y);
+          }
         }
         uint8_t* row;
         int chunk0;
@@ -595,7 +621,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             float v[16];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              hw[e] = pack_bf16x2(gelu(__uint_as_float(yw[e] << 16)), gelu(__uint_as_float(yw[e] & 0xFFFF0000u)));
+              hw[e] = gelu_bf16x2(yw[e]);
               v[2 * e] = __uint_as_float(hw[e] << 16);
               v[2 * e + 1] = __uint_as_float(hw[e] & 0xFFFF0000u);
             }
@@ -668,6 +694,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // T = bf16(t_scale * sum over the partial slots of each 256-row block, in slot
 // order); one thread per element, 8 rows per CTA.
 constexpr int kReduceRows = 8;
+constexpr int kReduceUnroll = 8;
 __global__ void mlp_t_reduce_kernel(const float* tpart, int M_pad, int slots, int n_tiles, int n_blocks, int n_pairs,
                                     float t_scale, __nv_bfloat16* T) {
   const int mp = blockIdx.x / (2 * kBM / kReduceRows);
@@ -680,8 +707,18 @@ __global__ void mlp_t_reduce_kernel(const float* tpart, int M_pad, int slots, in
   const int used = used_s;
   if (m >= M_pad) return;
   const float* src = tpart + (static_cast<size_t>(mp) * slots * (2 * kBM) + r) * kMlpDownRP + c;
+  const int n = used < slots ? used : slots;
+  // the slots' loads all in flight at once (up to kReduceUnroll), summed in slot order
   float acc = 0.f;
-  for (int sl = 0; sl < used && sl < slots; ++sl) acc += src[static_cast<size_t>(sl) * (2 * kBM) * kMlpDownRP];
+  for (int s0 = 0; s0 < n; s0 += kReduceUnroll) {
+    float v[kReduceUnroll];
+#pragma unroll
+    for (int u = 0; u < kReduceUnroll; ++u)
+      v[u] = s0 + u < n ? src[static_cast<size_t>(s0 + u) * (2 * kBM) * kMlpDownRP] : 0.f;
+#pragma unroll
+    for (int u = 0; u < kReduceUnroll; ++u)
+      if (s0 + u < n) acc += v[u];
+  }
   T[static_cast<size_t>(m) * kMlpDownRP + c] = __float2bfloat16_rn(acc * t_scale);
 }
 
