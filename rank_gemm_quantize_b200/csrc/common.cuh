@@ -284,7 +284,7 @@ constexpr uint32_t kFmtE4M3 = 0;  // A/B format code of E4M3 in kind::f8f6f4
 
 __device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8]) {
   uint32_t out;
-  asm volatile(
+  asm(  // pure conversions: no side effects, so the compiler may schedule them freely
       "{\n .reg .b8 b0, b1, b2, b3;\n"
       " cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n"
       " cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n"
@@ -299,14 +299,14 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8]) {
 // Two floats -> two E4M3 bytes (lo in bits 7:0, hi in bits 15:8).
 __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
   uint16_t out;
-  asm volatile("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(hi), "f"(lo));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(hi), "f"(lo));
   return out;
 }
 
 __device__ __forceinline__ float e4m3_to_float(uint32_t byte) {
   uint32_t h2;
   uint16_t in = static_cast<uint16_t>(byte & 0xFF);
-  asm volatile("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
   return __half2float(__ushort_as_half(static_cast<uint16_t>(h2 & 0xFFFF)));
 }
 

@@ -180,27 +180,23 @@ __device__ __forceinline__ TileRange tile_range(int pair, int n_pairs, int n_til
   return {pair, n_tiles, n_pairs};
 }
 
-// The first pair whose contiguous range holds a tile of 256-row block mp: the
-// smallest p with floor((p + 1) n_tiles / n_pairs) > t for the block's first
-// tile t, i.e. p = ceil((t + 1) n_pairs / n_tiles) - 1.
-__host__ __device__ inline int mlp_first_pair(int mp, int n_blocks, int n_tiles, int n_pairs) {
-  const long long t = static_cast<long long>(mp) * n_blocks;
-  const long long p = ((t + 1) * n_pairs + n_tiles - 1) / n_tiles - 1;
-  return static_cast<int>(p < 0 ? 0 : (p > n_pairs - 1 ? n_pairs - 1 : p));
+// Pair p takes tiles [floor(p T / P), floor((p + 1) T / P)) of the T tiles
+// (P <= T pairs, so no range is empty). The pair holding tile t is the
+// smallest p with floor((p + 1) T / P) > t, i.e. p = ceil((t + 1) P / T) - 1.
+// The host keeps T P below 2^31, so the products fit in 32 bits.
+__host__ __device__ inline int mlp_pair_of_tile(int t, int n_tiles, int n_pairs) {
+  const int p = ((t + 1) * n_pairs + n_tiles - 1) / n_tiles - 1;
+  return p < 0 ? 0 : (p > n_pairs - 1 ? n_pairs - 1 : p);
 }
-
+// The first pair whose range holds a tile of 256-row block mp.
+__host__ __device__ inline int mlp_first_pair(int mp, int n_blocks, int n_tiles, int n_pairs) {
+  return mlp_pair_of_tile(mp * n_blocks, n_tiles, n_pairs);
+}
 // The number of pairs whose ranges hold tiles of row block mp (the partial
-// slots it uses).
+// slots it uses): from the pair of its first tile to the pair of its last.
 __host__ __device__ inline int mlp_block_pairs(int mp, int n_blocks, int n_tiles, int n_pairs) {
-  const long long t0 = static_cast<long long>(mp) * n_blocks, t1 = t0 + n_blocks;
-  int used = 0;
-  for (int pp = mlp_first_pair(mp, n_blocks, n_tiles, n_pairs); pp < n_pairs; ++pp) {
-    const long long f = (static_cast<long long>(pp) * n_tiles) / n_pairs;
-    const long long l = (static_cast<long long>(pp + 1) * n_tiles) / n_pairs;
-    if (f >= t1) break;
-    if (l > t0 && l > f) ++used;
-  }
-  return used;
+  return mlp_pair_of_tile(mp * n_blocks + n_blocks - 1, n_tiles, n_pairs) -
+         mlp_pair_of_tile(mp * n_blocks, n_tiles, n_pairs) + 1;
 }
 
 template <bool kMlp>
@@ -601,38 +597,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
       if (kMlp) {
-        // Phase B, overlapping the next tile's mainloop: h = bf16(GELU(y)) in place, then the down
-        // layer's smoothing and NVFP4 groups of 16; this thread's row, 64 columns at a time
+        // Phase B, overlapping the next tile's mainloop. B1: h = bf16(GELU(y)) in place over this
+        // thread's row slice; then the T contraction may read h (the fence comes before any of this
+        // tile's global stores, so it does not wait for them). B2: the down layer's smoothing and
+        // NVFP4 groups of 16 from the staged h.
         const float* is_tile = reinterpret_cast<const float*>(smem + L::kIsOff + bs * L::kIs);
         const int m = row0 + lane;
+        uint8_t* hrow = smem + L::kStgOff + (col0 >> 6) * L::kHChunk + rc * 128;
+#pragma unroll
+        for (int piece = 0; piece < kEpiCols / 64; ++piece) {
+#pragma unroll
+          for (int c16 = 0; c16 < 8; ++c16) {  // 16-byte chunk of the 128-byte row (8 values)
+            uint4* pc = reinterpret_cast<uint4*>(hrow + piece * L::kHChunk + ((c16 ^ (rc & 7)) << 4));
+            const uint4 u = *pc;
+            *pc = make_uint4(gelu_bf16x2(u.x), gelu_bf16x2(u.y), gelu_bf16x2(u.z), gelu_bf16x2(u.w));
+          }
+        }
+        fence_proxy_async_smem();  // h is read by the T contraction's MMAs
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(h_ready, 0);
 #pragma unroll 1
         for (int piece = 0; piece < kEpiCols / 64; ++piece) {
           const int cn = col0 + 64 * piece;  // first column of the 64 within the tile
-          uint8_t* row = smem + L::kStgOff + (cn >> 6) * L::kHChunk + rc * 128;
+          const uint8_t* row = hrow + piece * L::kHChunk;
           uint32_t cw[8];
           uint32_t sbw = 0;
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
-            uint4* p0 = reinterpret_cast<uint4*>(row + (((2 * g) ^ (rc & 7)) << 4));
-            uint4* p1 = reinterpret_cast<uint4*>(row + (((2 * g + 1) ^ (rc & 7)) << 4));
-            const uint4 u0 = *p0, u1 = *p1;
-            const uint32_t yw[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-            uint32_t hw[8];
+            const uint4 u0 = *reinterpret_cast<const uint4*>(row + (((2 * g) ^ (rc & 7)) << 4));
+            const uint4 u1 = *reinterpret_cast<const uint4*>(row + (((2 * g + 1) ^ (rc & 7)) << 4));
+            const uint32_t hw[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
             float v[16];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              hw[e] = gelu_bf16x2(yw[e]);
-              v[2 * e] = __uint_as_float(hw[e] << 16);
-              v[2 * e + 1] = __uint_as_float(hw[e] & 0xFFFF0000u);
-            }
-            *p0 = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-            *p1 = make_uint4(hw[4], hw[5], hw[6], hw[7]);
             const float* is = is_tile + cn + 16 * g;
 #pragma unroll
             for (int e = 0; e < 16; e += 4) {
               const float4 s4 = *reinterpret_cast<const float4*>(is + e);
-              const float2 a = __fmul2_rn(make_float2(v[e], v[e + 1]), make_float2(s4.x, s4.y));
-              const float2 b2 = __fmul2_rn(make_float2(v[e + 2], v[e + 3]), make_float2(s4.z, s4.w));
+              const float2 a = __fmul2_rn(make_float2(__uint_as_float(hw[e / 2] << 16),
+                                                      __uint_as_float(hw[e / 2] & 0xFFFF0000u)),
+                                          make_float2(s4.x, s4.y));
+              const float2 b2 = __fmul2_rn(make_float2(__uint_as_float(hw[e / 2 + 1] << 16),
+                                                       __uint_as_float(hw[e / 2 + 1] & 0xFFFF0000u)),
+                                           make_float2(s4.z, s4.w));
               v[e] = a.x;
               v[e + 1] = a.y;
               v[e + 2] = b2.x;
@@ -650,12 +655,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint32_t*>(mlp.scales + atom * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4) = sbw;
           }
         }
-        fence_proxy_async_smem();  // h is read by the T contraction's MMAs
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&is_empty[bs]);
-          mbar_arrive_cluster(h_ready, 0);
-        }
+        if (lane == 0) mbar_arrive(&is_empty[bs]);
       }
       // MLP: the previous tile closed a row block: its partial is complete (its
       // contraction was committed before this tile's accumulator)
@@ -701,10 +702,7 @@ __global__ void mlp_t_reduce_kernel(const float* tpart, int M_pad, int slots, in
   const int r = (blockIdx.x % (2 * kBM / kReduceRows)) * kReduceRows + threadIdx.x / kMlpDownRP;
   const int c = threadIdx.x % kMlpDownRP;
   const int m = mp * 2 * kBM + r;
-  __shared__ int used_s;  // pairs whose range holds a tile of this block
-  if (threadIdx.x == 0) used_s = mlp_block_pairs(mp, n_blocks, n_tiles, n_pairs);
-  __syncthreads();
-  const int used = used_s;
+  const int used = mlp_block_pairs(mp, n_blocks, n_tiles, n_pairs);  // pairs whose range holds a tile of this block
   if (m >= M_pad) return;
   const float* src = tpart + (static_cast<size_t>(mp) * slots * (2 * kBM) + r) * kMlpDownRP + c;
   const int n = used < slots ? used : slots;

@@ -842,6 +842,8 @@ svdq_status mlp_impl(svdq_layer* up, svdq_layer* down, const void* X, int M, voi
     return fail(SVDQ_ERR_INVALID_ARG, "X/Y must be 16-byte and the workspace 256-byte aligned");
   if (svdq_status e = check_layer_device(up)) return e;
   const MlpLayout l = mlp_layout(up, down, M);
+  if (static_cast<long long>(l.tiles + 1) * l.pairs >= (1LL << 31))
+    return fail(SVDQ_ERR_INVALID_ARG, "M exceeds the rows the fused MLP block supports");
   if (ws_bytes < l.total) return fail(SVDQ_ERR_INVALID_ARG, "workspace too small");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(workspace);
