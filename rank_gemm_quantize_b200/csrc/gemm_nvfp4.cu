@@ -52,7 +52,7 @@
 // the down layer's branch input T. A pair takes a contiguous range of tiles
 // in row-major tile order, so T accumulates over the pair's tiles of one
 // 256-row block; it is flushed as a float partial when the row block changes
-// and the partials are summed in a fixed order by nvfp4_mlp_t_reduce. The
+// and the partials are summed in a fixed order by mlp_t_reduce_kernel. The
 // contraction of tile i is issued after the next tile's mainloop MMAs, so it
 // overlaps the epilogue instead of waiting for it.
 #include <cstdint>

@@ -84,7 +84,7 @@ struct GemmMaps {
 // NVFP4 GEMM sees it: GELU of the up output is smoothed and quantized
 // straight into the down layer's activation buffers, and its branch input T
 // is accumulated from the same tile (partials over the pairs of SMs, summed
-// by nvfp4_mlp_t_reduce).
+// by mlp_t_reduce_kernel).
 constexpr int kMlpDownRP = 32;  // branch width of the down layer the fused epilogue supports
 struct MlpDownParams {
   int K;                 // the down layer's K (= the up layer's N)
