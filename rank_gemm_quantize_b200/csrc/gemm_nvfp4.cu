@@ -32,12 +32,13 @@
 //           commits free the stage in both CTAs and mark the tile;
 //   warps 2-17 epilogue (both), four per TMEM lane quarter (enough warps to
 //           hide the latency of the MLP variant's per-element work): each
-//           reads its 32 rows x 64 columns of its
-//           CTA's accumulator 32 columns at a time, scales, adds the bias,
-//           packs bf16 and writes it into a 128-byte-swizzled staging buffer
-//           right away; then it tells the leader that TMEM is free (the next
-//           tile's MMAs start) and stores its 32 x 64 box with TMA
-//           (rows and columns past M and N are clipped by the tensor map).
+//           reads its 32 rows x 64 columns of its CTA's accumulator 32
+//           columns at a time, scales, adds the bias and packs bf16; after
+//           the last TMEM load it tells the leader that TMEM is free (the
+//           next tile's MMAs start). Each 32 x 32 chunk goes through the
+//           warp's one 2 KB staging box (64-byte swizzle) and out with a TMA
+//           store (rows and columns past M and N are clipped by the tensor
+//           map); the small staging leaves shared memory for a fifth stage.
 //
 // MLP-block variant (kMlp, the up layer of up -> GELU -> down): the branch
 // reads T as a bf16 pair (T + T_lo, about 16 significant bits), so the up
@@ -75,7 +76,7 @@ constexpr int kThreads = (3 + kEpiWarps) * 32;
 
 template <bool kMlp>
 struct SmemNv {
-  static constexpr int kStages = kMlp ? 3 : 4;
+  static constexpr int kStages = kMlp ? 3 : 5;
   static constexpr int kA = kBM * kBKBytes;       // 16 KB
   static constexpr int kB = kBNHalf * kBKBytes;   // 16 KB
   static constexpr int kSfa = 4 * 512;            // this CTA's 128 rows, 4 k-blocks of 64
@@ -86,9 +87,10 @@ struct SmemNv {
   // Y staging for the TMA stores (16 warps x one 32 x 64 box); in the MLP
   // variant the same 64 KB hold h as four K-major 128 x 64 bf16 chunks.
   static constexpr int kStgOff = kBiasOff + 2 * kBias;
-  static constexpr int kStgBox = 32 * 128;
-  static constexpr int kStgWarp = (kEpiCols / 64) * kStgBox;
-  static constexpr int kStg = kEpiWarps * kStgWarp;  // 64 KB
+  // Y staging (plain): one 32 x 32 box per epilogue warp (2 KB, 64-byte swizzle), reused
+  // chunk after chunk; in the MLP variant the 64 KB hold h as four K-major 128 x 64 chunks.
+  static constexpr int kStgWarp = 32 * 64;
+  static constexpr int kStg = kMlp ? 4 * kBM * 128 : kEpiWarps * kStgWarp;  // 64 KB / 32 KB
   static constexpr int kHChunk = kBM * 128;          // 16 KB: 128 rows x 64 bf16
   static constexpr int kIsOff = kStgOff + kStg;      // MLP: down-layer inv_s slices, 2 x 256 floats
   static constexpr int kIs = kMlp ? kBN * 4 : 0;
@@ -542,15 +544,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const uint4* bias4 = reinterpret_cast<const uint4*>(smem + L::kBiasOff + bs * L::kBias) + col0 / 8;
-      if (!kMlp) {
-        if (lane == 0) bulk_wait_group_read<0>();  // this warp's previous stores have read the staging boxes
-        __syncwarp();
-      }
       const uint32_t ta = tmem + (static_cast<uint32_t>(32 * q) << 16) + col0;
-      // Phase A: the accumulator -> y = out_scale acc + b, bf16, into the staging buffer (the Y
-      // boxes; in the MLP block the K-major h chunks, where phase B turns y into h in place)
+      // Phase A: the accumulator -> y = out_scale acc + b, bf16. Plain: into this warp's 32 x 32
+      // staging box and out with a TMA store, 32 columns at a time; MLP block: into the K-major
+      // h chunks, where phase B turns y into h in place.
 #pragma unroll
-      for (int c = 0; c < kEpiCols / 32; ++c) {  // 32 columns: half of one 64-column staging box
+      for (int c = 0; c < kEpiCols / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(ta + 32 * c, r);
         tmem_ld_wait();
@@ -567,33 +566,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             o[4 * v + e] = pack_bf16x2(yv.x, yv.y);
           }
         }
-        uint8_t* row;
-        int chunk0;
+        if (c == kEpiCols / 32 - 1) {
+          // every load of the tile has landed: this CTA's share of TMEM is free, the next tile's
+          // MMAs start; the bias slot is free too
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive_cluster(acc_empty, 0);
+            mbar_arrive(&bias_empty[bs]);
+          }
+        }
         if (!kMlp) {
-          row = stg + (c >> 1) * L::kStgBox + lane * 128;
-          chunk0 = 4 * (c & 1);
+          if (lane == 0) bulk_wait_group_read<0>();  // the previous store has read the box
+          __syncwarp();
+          uint8_t* row = stg + lane * 64;  // 64-byte rows, 16-byte chunk j at j ^ ((row / 2) % 4)
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            *reinterpret_cast<uint4*>(row + ((v ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&maps.y, stg, nb * kBN + col0 + 32 * c, row0);
+            bulk_commit_group();
+          }
         } else {
           const int cn = col0 + 32 * c;
-          row = smem + L::kStgOff + (cn >> 6) * L::kHChunk + rc * 128;
-          chunk0 = (cn & 63) >> 3;
-        }
-        const int sw = kMlp ? (rc & 7) : (lane & 7);
+          uint8_t* row = smem + L::kStgOff + (cn >> 6) * L::kHChunk + rc * 128;
+          const int chunk0 = (cn & 63) >> 3;
 #pragma unroll
-        for (int v = 0; v < 4; ++v)
-          *reinterpret_cast<uint4*>(row + (((chunk0 + v) ^ sw) << 4)) =
-              make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
-      }
-      tc_fence_before();
-      if (!kMlp) fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_cluster(acc_empty, 0);  // this CTA's share of TMEM is free: the next tile's MMAs start
-        mbar_arrive(&bias_empty[bs]);
-        if (!kMlp) {
-#pragma unroll
-          for (int b = 0; b < kEpiCols / 64; ++b)
-            tma_store_2d(&maps.y, stg + b * L::kStgBox, nb * kBN + col0 + 64 * b, row0);
-          bulk_commit_group();
+          for (int v = 0; v < 4; ++v)
+            *reinterpret_cast<uint4*>(row + (((chunk0 + v) ^ (rc & 7)) << 4)) =
+                make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
         }
       }
       if (kMlp) {

@@ -74,7 +74,7 @@ struct GemmMaps {
   CUtensorMap l2;   // L2T [N_pad, RP] bf16
   CUtensorMap sfa;  // NVFP4 activation scale-factor atoms as uint32 [atoms, 128], box {128, 4}
   CUtensorMap sfb;  // NVFP4 weight scale-factor atoms, same view
-  CUtensorMap y;    // NVFP4: Y [M, N] bf16, box {64, 32}, 128-byte swizzle (TMA stores)
+  CUtensorMap y;    // NVFP4: Y [M, N] bf16, box {32, 32}, 64-byte swizzle (TMA stores)
   CUtensorMap l1h_down;  // MLP block: the down layer's L1s^T high part [RP_down, K_down], box {64, RP_down / 2}
   CUtensorMap l1l_down;  // ... and low part
   CUtensorMap t_lo;      // MLP block: the up layer's T low part [M_pad, RP] bf16, as t

@@ -755,8 +755,8 @@ svdq_status gemm_stage(svdq_layer* h, int M, void* Y, uint8_t* codes, void* scal
     auto* ye = h->y_maps.find(Y, M);
     if (!ye) {
       ye = h->y_maps.insert(Y, M);
-      if (!make_map(&ye->a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, h->N, M, static_cast<uint64_t>(h->N) * 2, 64, 32,
-                    CU_TENSOR_MAP_SWIZZLE_128B)) {
+      if (!make_map(&ye->a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, h->N, M, static_cast<uint64_t>(h->N) * 2, 32, 32,
+                    CU_TENSOR_MAP_SWIZZLE_64B)) {
         ye->key = nullptr;
         return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (Y) failed");
       }
