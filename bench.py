@@ -63,7 +63,8 @@ def workload_desc(cfg: int, layers, fused: bool = False) -> str:
         return (f"FLUX-like MLP pair: up [{L.M},{L.K}]x[{L.K},{L.N}] then down [{L.M},{layers[1].K}]x"
                 f"[{layers[1].K},{layers[1].N}], rank {L.rank}, {L.fmt}")
     if cfg == 4:
-        return f"sweep point K=N=3072, M={L.M}, rank {L.rank}, {L.fmt}"
+        lora = "" if L.lora_A is None else f" + a rank-{L.lora_A.shape[1]} LoRA in the branch"
+        return f"sweep point K=N=3072, M={L.M}, rank {L.rank}{lora}, {L.fmt}"
     return f"single linear [{L.M},{L.K}]x[{L.K},{L.N}], rank {L.rank}, {L.fmt}"
 
 
@@ -92,8 +93,17 @@ def load_layers(args):
         kw["rank"] = args.rank
     if args.fmt:
         kw["fmt"] = args.fmt
+    if getattr(args, "lora", False):
+        if args.config != 4:
+            raise SystemExit("--lora belongs to the sweep (--config 4)")
+        kw["lora"] = True
     layers = workloads.config(args.config, **kw)
     return layers
+
+
+def branch_rank(L) -> int:
+    """Columns of the layer's low-rank branch: its rank plus an attached adapter's."""
+    return L.rank + (0 if L.lora_A is None else int(L.lora_A.shape[1]))
 
 
 # A timed region shorter than this is a burst: the clocks have not settled
@@ -143,7 +153,8 @@ def config_dict(args, layers) -> dict:
     n_sets, set_bytes = rotation_sets(layers, fused)
     L = layers[0]
     return {"workload": workload_desc(args.config, layers, fused), "config_id": args.config,
-            "M": L.M, "K": L.K, "N": L.N, "rank": L.rank, "format": L.fmt, "layers_per_step": len(layers),
+            "M": L.M, "K": L.K, "N": L.N, "rank": L.rank, "lora_rank": branch_rank(L) - L.rank, "format": L.fmt,
+            "layers_per_step": len(layers),
             "pipeline": ("fused MLP block (activation kernel, up GEMM with GELU and the down layer's quantization "
                          "in its epilogue, T sum, down GEMM)" if fused else "one forward per layer"),
             "l2": f"inputs larger than L2: {n_sets} rotating sets of prepared layer + X/Y/workspace "
@@ -309,7 +320,9 @@ def run_ours(args):
             X0 = L.X.to(dev)
             a = rq.calibrate_absmax(X0)
         g0 = rq.Layer.prepare(L.W.to(dev), L.bias.to(dev), a, L.fmt, L.rank, alpha=L.alpha)
-        ex = g0.export()
+        ex = g0.export()  # the prepared layer's own factors, before any adapter
+        if L.lora_A is not None:
+            g0.attach_lora(L.lora_A.to(dev), L.lora_B.to(dev), L.lora_scale)
         preps.append((L, X0, a, g0, ex))
     n_sets, _ = rotation_sets(layers, fused)
     sets = []
@@ -322,6 +335,8 @@ def run_ours(args):
                 L1 = torch.from_numpy(ex["L1"]).to(torch.bfloat16).to(dev)
                 L2 = torch.from_numpy(ex["L2"]).to(torch.bfloat16).to(dev)
                 g = rq.Layer.prepare(L.W.to(dev), L.bias.to(dev), a, L.fmt, L.rank, alpha=L.alpha, factors=(L1, L2))
+                if L.lora_A is not None:
+                    g.attach_lora(L.lora_A.to(dev), L.lora_B.to(dev), L.lora_scale)
             X = None if X0 is None else (X0 if s == 0 else X0.clone())
             Y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device=dev) if not fused or L is layers[-1] else None
             ws = None if fused else torch.empty(g.workspace_size(L.M), dtype=torch.uint8, device=dev)
@@ -390,7 +405,7 @@ def run_ours(args):
         reduce_ms = None
     max_ms = max_over_ranks(elapsed_ms, world, dev)
 
-    step_ops = sum(layer_ops(L.M, L.K, L.N, L.rank) for L in layers)
+    step_ops = sum(layer_ops(L.M, L.K, L.N, branch_rank(L)) for L in layers)
     value = whole_job_tops(step_ops, K_steps, world, max_ms)
     ms_per_step = max_ms / K_steps
 
@@ -512,7 +527,7 @@ def run_ours(args):
     # ---- roofline of the dominant kernel (the GEMM) and of the activation kernel
     fmt = layers[0].fmt
     wl_key = f"cfg{args.config}_M{layers[0].M}_r{layers[0].rank}_{fmt}" + ("_fused" if fused else "")
-    g_ops = sum(gemm_ops(L.M, L.K, L.N, L.rank) for L in layers)
+    g_ops = sum(gemm_ops(L.M, L.K, L.N, branch_rank(L)) for L in layers)
     g_s = sum(gemm_ms) * 1e-3
     tensor_peak, peak_desc = tensor_peak_for(peaks, fmt, elapsed_ms * 1e-3)
     gemm_name = "gemm_int4_kernel" if fmt == "int4_g64" else "gemm_nvfp4_kernel"
@@ -522,7 +537,7 @@ def run_ours(args):
                 "traffic": traffic,
                 "peak_source": f"{peak_kind} {peak_desc}",
                 "algorithmic": "2MKN + 2MrN per launch", "frac_of_datasheet_dense": g_ops / g_s / 1e12 / DATASHEET_TOPS[fmt]}
-    k_bytes = sum(k1_bytes(L.M, L.K, L.rank, fmt) for L in (layers[:1] if fused else layers))
+    k_bytes = sum(k1_bytes(L.M, L.K, branch_rank(L), fmt) for L in (layers[:1] if fused else layers))
     k_s = sum(k1_ms) * 1e-3
     k1_roof = {"bound": "hbm", "kernel": "act_quant_kernel", "achieved": k_bytes / k_s / 1e9, "peak": peaks["hbm_gbs"],
                "unit": "GB/s", "frac": k_bytes / k_s / 1e9 / peaks["hbm_gbs"],
@@ -640,6 +655,8 @@ def _oracle_prepare(layers):
         X = workloads.to_f64(L.X)
         a = S.calibrate_absmax(X)
         p = S.prepare(workloads.to_f64(L.W), workloads.to_f64(L.bias), a, L.fmt, L.alpha, L.rank)
+        if L.lora_A is not None:
+            p = S.attach_lora(p, workloads.to_f64(L.lora_A), workloads.to_f64(L.lora_B), L.lora_scale)
         S.dequantized_weight(p)
         out.append((L, X, p))
     return out
@@ -669,7 +686,7 @@ def cpu_baseline(layers, budget_s: float = 10.0, rows=None):
             S.forward(p, X[:r])
         t_total += time.perf_counter() - t
         n += 1
-        ops += sum(layer_ops(r, L.K, L.N, L.rank) for L in layers)
+        ops += sum(layer_ops(r, L.K, L.N, branch_rank(L)) for L in layers)
         if t_total >= budget_s or n >= 50:
             break
     return {"value": ops / t_total / 1e12, "unit": "TOPS", "cores": _blas_threads(), "kind": "oracle",
@@ -694,7 +711,7 @@ def run_reference(args):
         for (L, X, p) in preps:
             S.forward(p, X[:rows])
     dt = time.perf_counter() - t
-    ops = sum(layer_ops(rows, L.K, L.N, L.rank) for L in layers) * args.steps
+    ops = sum(layer_ops(rows, L.K, L.N, branch_rank(L)) for L in layers) * args.steps
     value = ops / dt / 1e12
     fmt = layers[0].fmt
     cores = _blas_threads()
@@ -727,6 +744,7 @@ def parse_args(argv=None):
     ap.add_argument("--unfused", action="store_true",
                     help="run an NVFP4 MLP pair as two layer forwards instead of the fused MLP block")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--lora", action="store_true", help="sweep (--config 4) with a rank-32 LoRA in the branch")
     ap.add_argument("--ablation", action="store_true",
                     help="print the error / time table of the method's ablations instead of the benchmark line")
     return ap.parse_args(argv)
