@@ -110,14 +110,15 @@ static_assert(kBNHalf == kWeightBoxRows && kBM == kActBoxRows, "each CTA loads o
 // TMEM columns (each CTA): accumulator [0, 256), then one scale-factor slot per
 // shared-memory stage (A: 16 columns, B: 32), so copying the next k-tile's
 // scale factors never waits for the MMAs still reading the previous ones;
-// then (MLP) the down layer's T accumulator.
+// then (MLP) the down layer's T accumulator (64 columns: the products with the
+// factor's high and low bf16 parts side by side, summed when read out).
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfSlotCols = 16 + 2 * 16;
 constexpr uint32_t kSfaCol = kBN;
 constexpr uint32_t kSfbCol = kBN + 16;
 template <bool kMlp>
 constexpr uint32_t t_acc_col() { return kBN + SmemNv<kMlp>::kStages * kSfSlotCols; }
-static_assert(t_acc_col<true>() + kMlpDownRP <= kTmemCols && t_acc_col<false>() <= kTmemCols, "TMEM budget");
+static_assert(t_acc_col<true>() + 2 * kMlpDownRP <= kTmemCols && t_acc_col<false>() <= kTmemCols, "TMEM budget");
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -380,7 +381,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (leader) {
       const uint32_t idesc_main = idesc_block_scaled(2 * kBM, kBN);
       const uint32_t idesc_lr = idesc_dense(kFmtF32, kFmtBF16, kFmtBF16, 2 * kBM, kBN);
-      const uint32_t idesc_t = idesc_dense(kFmtF32, kFmtBF16, kFmtBF16, 2 * kBM, kMlpDownRP);
+      // T contraction: N = 64, each CTA's 32 B rows being its 16 ranks of L1s^T's high part, then
+      // the same 16 ranks' low part (adjacent in the slot), so one MMA takes both
+      const uint32_t idesc_t = idesc_dense(kFmtF32, kFmtBF16, kFmtBF16, 2 * kBM, 2 * kMlpDownRP);
       bool ok = true;
       int it = 0, ti = 0;
       int flushes = 0;  // MLP: row-block partials of T flushed so far
@@ -400,13 +403,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 4; ++c)
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              const uint64_t ad = smem_desc(hst + c * L::kHChunk + 32 * ks, 16, 1024, kSw128);
-              mma_f16_pair(tacc, ad, smem_desc(l1 + (2 * c) * L::kL1Part + 32 * ks, 16, 1024, kSw128), idesc_t,
+            for (int ks = 0; ks < 4; ++ks)
+              mma_f16_pair(tacc, smem_desc(hst + c * L::kHChunk + 32 * ks, 16, 1024, kSw128),
+                           smem_desc(l1 + (2 * c) * L::kL1Part + 32 * ks, 16, 1024, kSw128), idesc_t,
                            (first && c == 0 && ks == 0) ? 0u : 1u);
-              mma_f16_pair(tacc, ad, smem_desc(l1 + (2 * c + 1) * L::kL1Part + 32 * ks, 16, 1024, kSw128), idesc_t,
-                           1u);
-            }
           tc_commit_pair_mc(&l1_empty[j & 1], 0x3);
           if (last) tc_commit_pair_mc(t_full, 0x3);
         }
@@ -519,15 +519,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int mp = tile_j / n_blocks;
       const int slot = pair - mlp_first_pair(mp, n_blocks, n_tiles, n_pairs);
-      uint32_t r[32];
-      tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + t_acc_col<kMlp>(), r);
-      tmem_ld_wait();
       float* dst = mlp.tpart + ((static_cast<size_t>(mp) * mlp.slots + slot) * (2 * kBM) +
                                 static_cast<int>(rank) * kBM + rc) * kMlpDownRP;
+      // accumulator columns: [16 ranks high | the same ranks low] per CTA half of the pair
 #pragma unroll
-      for (int e = 0; e < kMlpDownRP; e += 4)
-        *reinterpret_cast<float4*>(dst + e) = make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
-                                                          __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+      for (int half = 0; half < 2; ++half) {
+        uint32_t r[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + t_acc_col<kMlp>() + 32 * half, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; e += 4)
+          *reinterpret_cast<float4*>(dst + 16 * half + e) =
+              make_float4(__uint_as_float(r[e]) + __uint_as_float(r[e + 16]),
+                          __uint_as_float(r[e + 1]) + __uint_as_float(r[e + 17]),
+                          __uint_as_float(r[e + 2]) + __uint_as_float(r[e + 18]),
+                          __uint_as_float(r[e + 3]) + __uint_as_float(r[e + 19]));
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(t_empty, 0);
